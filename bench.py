@@ -1,0 +1,485 @@
+"""Benchmark of the decode-time QSA hot path on B200.
+
+One step = compress-append of the new token(s) + indexer top-k over every
+micro-block + sparse split-KV decode over the selected tokens + LSE merge,
+for one batch of the named workload (default: batch 128 x 262,144-token
+contexts, GQA 16/2, D 128, bf16, 2 KV splits).  The caches (K/V, compressed
+keys) are built untimed and stay resident; the compressed-key scan alone
+(2 GiB per step) is far larger than L2, so no flush is needed between steps.
+
+Prints ONE JSON line on rank 0.  ``--impl reference`` times the CPU oracle
+(the reference arm of this method: there is no runnable reference code) on
+a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QSA decode queries/s and achieved HBM GB/s (% of B200 peak) at 256k ctx"
+UNIT = "queries/s"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="b128_256k")
+    ap.add_argument("--splits", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-queries", type=int, default=8,
+                    help="oracle queries timed for the CPU baseline")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic bytes (what the method must move), per query and per launch
+# ---------------------------------------------------------------------------
+
+def algorithmic_bytes(w, L: int, num_splits: int) -> dict:
+    """Bytes one query (one request, T query tokens) must move.
+
+    index_topk : every competing compressed key (int16, d per block), the
+                 block-table entries of those pages, the indexer query and
+                 the selection row written.
+    sparse_decode : K and V rows of the selected tokens for every kv head,
+                 the query, the block-table entries of the selected pages
+                 (counted once per page of the table row already), the
+                 partial outputs written.
+    lse_merge  : partial outputs read, merged output written.
+    """
+    n = (L - w.T) // 4 + 1
+    P = w.page_size
+    kv_elem = {"f32": 4, "bf16": 2, "e4m3": 1}[w.kv_dtype]
+    q_elem = {"f32": 4, "bf16": 2}[w.q_dtype]
+    pages = math.ceil(n * 4 / P)
+    topk = min(w.topk, n)
+    tokens = topk * 4 + (w.T - 1)
+    idx = n * w.d_idx * 2 + pages * 4 + w.d_idx + w.topk * 4
+    dec = (2 * tokens * w.Hkv * w.D * kv_elem + w.T * w.Hq * w.D * q_elem + w.topk * 4
+           + num_splits * w.T * w.Hq * (w.D + 1) * 4)
+    if w.kv_dtype == "e4m3":
+        dec += 2 * min(tokens, math.ceil(L / P)) * w.Hkv * 4
+    merge = num_splits * w.T * w.Hq * (w.D + 1) * 4 + w.T * w.Hq * (w.D + 1) * 4
+    append = w.T * w.d_idx * 3 + 2 * w.d_idx * 2
+    return dict(index_topk=idx, sparse_decode=dec, lse_merge=merge, compress_append=append,
+                total=idx + dec + merge + append)
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
+    return dict(hbm_gbs=6650.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+
+REASON_KEYS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={q}", "--format=csv,noheader",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def mark(self, which: str):
+        setattr(self, which, time.time())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                sm = float(parts[1].split()[0])
+                smax = float(parts[2].split()[0])
+            except (ValueError, IndexError):
+                continue
+            flags = {k: parts[5 + i].strip() == "Active" for i, k in enumerate(REASON_KEYS)}
+            rows.append((ts, sm, smax, flags))
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.06 <= r[0] <= self.t1 + 0.06]
+        use = inside if inside else rows
+        reasons = sorted({k for r in use for k, v in r[3].items() if v})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use),
+                "window": "timed region" if inside else "whole run"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_request_inputs(w, L: int, seed: int):
+    """Logical inputs of one request on the host (same recipe as the device
+    generator, drawn on the CPU)."""
+    from workloads.qsa_inputs import make_batch
+    import numpy as np
+    from oracle import qsa_ref as ref
+    b = make_batch(w, "cpu", seed=seed, ctx_lens=[L])
+    k_idx = b.k_idx.numpy()
+    if b.k_cache.dtype.itemsize == 2:
+        kst = b.k_cache.view(__import__("torch").int16).numpy().view(np.uint16)
+        vst = b.v_cache.view(__import__("torch").int16).numpy().view(np.uint16)
+        kind = "bf16"
+    elif b.k_cache.dtype.itemsize == 1:
+        kst = b.k_cache.view(__import__("torch").uint8).numpy()
+        vst = b.v_cache.view(__import__("torch").uint8).numpy()
+        kind = "e4m3"
+    else:
+        kst, vst, kind = b.k_cache.numpy(), b.v_cache.numpy(), "f32"
+    table = b.block_table_host[0].numpy()
+    K = ref.StoredRows(ref.depage(kst, table, L, w.page_size), kind,
+                       None if b.k_scale is None else b.k_scale.numpy()[table[np.arange(L) // w.page_size]])
+    V = ref.StoredRows(ref.depage(vst, table, L, w.page_size), kind,
+                       None if b.v_scale is None else b.v_scale.numpy()[table[np.arange(L) // w.page_size]])
+    qb = b.q[0]
+    if qb.dtype.itemsize == 2:
+        q = ref.bf16_bits_to_f64(qb.view(__import__("torch").int16).numpy().view(np.uint16))
+    else:
+        q = qb.double().numpy()
+    kc = ref.compress_keys(k_idx[: L - w.T])       # cache state before the step (untimed)
+    return dict(k_idx=k_idx, q_idx=b.q_idx[0].numpy(), q=q, K=K, V=V, kc_prefix=kc, L=L)
+
+
+def oracle_step(w, inp: dict, num_splits: int):
+    """One decode step of the oracle for one request, in the order of the GPU
+    step: compress the blocks the new tokens touch, score, select, attend
+    per split, merge."""
+    import numpy as np
+    from oracle import qsa_ref as ref
+    L, T = inp["L"], w.T
+    p0 = L - T
+    b0 = p0 // 4
+    touched = ref.compress_keys(inp["k_idx"][4 * b0: L])
+    kc = np.concatenate([inp["kc_prefix"][:b0], touched])
+    n_sel = ref.selection_width(L, T)
+    scores = ref.block_scores(inp["q_idx"], kc, n_sel)
+    sel = ref.select_blocks(scores, w.topk)
+    D = w.D
+    outs = []
+    for t in range(T):
+        toks = ref.token_set(sel, L, T, t)
+        op, lp = ref.split_attention(inp["q"][t], inp["K"], inp["V"], toks, 1.0 / math.sqrt(D), L,
+                                     w.page_size, num_splits)
+        outs.append(ref.lse_merge(op, lp))
+    return sel, outs
+
+
+_ORACLE_POOL: dict = {}
+
+
+def oracle_pool(w, n_distinct: int, seed: int) -> list:
+    """A few requests of workload w drawn on the host (cached; untimed)."""
+    from workloads.qsa_inputs import draw_ctx_lens
+    import torch
+    key = (w.name, n_distinct, seed)
+    if key not in _ORACLE_POOL:
+        lens = draw_ctx_lens(w, torch.Generator().manual_seed(seed)).tolist()
+        _ORACLE_POOL[key] = [oracle_request_inputs(w, int(lens[i % len(lens)]), seed + i)
+                             for i in range(n_distinct)]
+    return _ORACLE_POOL[key]
+
+
+def time_oracle(w, num_splits: int, n_queries: int, seed: int = 1000, n_distinct: int = 2) -> dict:
+    """Times the oracle (as it stands) on n_queries decode steps of workload
+    w, cycling over n_distinct host-drawn requests, on one host core; input
+    generation is not timed."""
+    from threadpoolctl import threadpool_limits
+    import torch
+    pool = oracle_pool(w, n_distinct, seed)
+    elapsed = 0.0
+    queries = 0
+    with threadpool_limits(limits=1):
+        nt = torch.get_num_threads()
+        torch.set_num_threads(1)
+        for i in range(n_queries):
+            inp = pool[i % len(pool)]
+            t0 = time.perf_counter()
+            oracle_step(w, inp, num_splits)
+            elapsed += time.perf_counter() - t0
+            queries += w.T
+        torch.set_num_threads(nt)
+    return dict(value=queries / elapsed, queries=queries, seconds=elapsed, cores=1,
+                distinct=len(pool))
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    from sparse_attention_decode_compress_b200 import (QSADecodeStep, qsa_get_device_error)
+    from sparse_attention_decode_compress_b200 import api as qapi
+    from workloads.qsa_inputs import WORKLOADS, make_batch
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload]
+    S = args.splits
+    batch = make_batch(w, dev, seed=w.seed + rank)
+    B, T = w.batch, w.T
+    L_host = batch.ctx_lens_host
+    max_blocks = int((L_host.max() + 3) // 4)
+
+    # caches (untimed): bulk append of all but the last T positions
+    cache = qapi.QSACache.allocate(batch.k_cache, batch.v_cache, batch.block_table, w.d_idx,
+                                   ring_rows=B, k_scale=batch.k_scale, v_scale=batch.v_scale)
+    n_pre = (L_host - T)
+    parts = [batch.k_idx[int(batch.cu_ctx_host[r]): int(batch.cu_ctx_host[r]) + int(n_pre[r])]
+             for r in range(B)]
+    k_pre = torch.cat(parts)
+    cu_pre = torch.zeros(B + 1, dtype=torch.int32)
+    cu_pre[1:] = torch.cumsum(n_pre, 0).to(torch.int32)
+    qapi.qsa_compress_append(cache, torch.zeros(B, dtype=torch.int32, device=dev), cu_pre.to(dev),
+                             k_pre, int(n_pre.max()))
+    del k_pre, parts
+    rows = torch.cat([torch.arange(int(batch.cu_ctx_host[r + 1]) - T, int(batch.cu_ctx_host[r + 1]))
+                      for r in range(B)]).to(dev)
+    k_new = batch.k_idx[rows].contiguous()
+    cu_new = torch.arange(0, B * T + 1, T, dtype=torch.int32, device=dev)
+    pos0 = (L_host - T).to(torch.int32).to(dev)
+    n_sel = ((L_host - T) // 4 + 1).to(torch.int32).to(dev) if T > 1 else None
+    step = QSADecodeStep(cache, B, T, w.Hq, w.topk, S, max_blocks)
+    stream = torch.cuda.current_stream()
+
+    def one_step(ev=None):
+        qapi.qsa_compress_append(cache, pos0, cu_new, k_new, T)
+        if ev is not None:
+            ev[0].record(stream)
+        qapi.qsa_index_topk(cache, batch.q_idx, batch.ctx_lens, n_sel, max_blocks, w.topk,
+                            step.sel, None, step.ws_topk)
+        if ev is not None:
+            ev[1].record(stream)
+        qapi.qsa_sparse_decode(cache, batch.q, batch.ctx_lens, step.sel, step.sm_scale, S,
+                               step.o_part, step.lse_part, step.ws_dec)
+        if ev is not None:
+            ev[2].record(stream)
+        qapi.qsa_lse_merge(step.o_part, step.lse_part, step.o, step.lse)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    st, flags = qsa_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error during warm-up: status {st} flags {flags}")
+
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark("t0")
+    t_start.record(stream)
+    for k in range(K):
+        one_step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark("t1")
+    if world > 1:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    topk_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    st, flags = qsa_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the timed region: status {st} flags {flags}")
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: t.cpu().pin_memory()
+        h_in = dict(pos0=pin(pos0), cu_new=pin(cu_new), k_new=pin(k_new), q_idx=pin(batch.q_idx),
+                    q=pin(batch.q), ctx_lens=pin(batch.ctx_lens))
+        if n_sel is not None:
+            h_in["n_sel"] = pin(n_sel)
+        d_in = {k: torch.empty_like(v, device=dev) for k, v in h_in.items()}
+        h_o = torch.empty(step.o.shape, dtype=torch.float32).pin_memory()
+        h_lse = torch.empty(step.lse.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in h_in.values())
+        d2h = h_o.numel() * 4 + h_lse.numel() * 4
+
+        def e2e_step():
+            for k_, v in h_in.items():
+                d_in[k_].copy_(v, non_blocking=True)
+            qapi.qsa_compress_append(cache, d_in["pos0"], d_in["cu_new"], d_in["k_new"], T)
+            qapi.qsa_index_topk(cache, d_in["q_idx"], d_in["ctx_lens"], d_in.get("n_sel"),
+                                max_blocks, w.topk, step.sel, None, step.ws_topk)
+            qapi.qsa_sparse_decode(cache, d_in["q"], d_in["ctx_lens"], step.sel, step.sm_scale, S,
+                                   step.o_part, step.lse_part, step.ws_dec)
+            qapi.qsa_lse_merge(step.o_part, step.lse_part, step.o, step.lse)
+            h_o.copy_(step.o, non_blocking=True)
+            h_lse.copy_(step.lse, non_blocking=True)
+
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        Ke = max(1, K // 2)
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * B * T * Ke / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    clocks = sampler.stop() if rank == 0 else None
+    if rank != 0:
+        return None
+
+    ab = [algorithmic_bytes(w, int(L), S) for L in L_host.tolist()]
+    idx_bytes = sum(a["index_topk"] for a in ab)
+    tot_bytes = sum(a["total"] for a in ab)
+    peaks = measured_peaks()
+    queries_per_step = B * T
+    value = world * queries_per_step * K / (ms / 1e3)
+    hbm = (tot_bytes * K / (ms / 1e3)) / 1e9
+    achieved = idx_bytes / (topk_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.kv_dtype if w.kv_dtype != "f32" else "f32",
+        "data": "synthetic (seeded; stands in for the pages' 256k-context serving trace)",
+        "config": {"workload": args.workload, "description": w.description, "global_batch": B * world,
+                   "seq_len": int(L_host.max()), "query_tokens": T, "kv_splits": S,
+                   "topk_blocks": w.topk, "page_size": w.page_size,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (2 GiB compressed keys read per step)"},
+        "hbm_gbs": round(hbm, 1),
+        "hbm_pct_of_peak": round(100 * hbm / peaks["hbm_gbs"], 2),
+        "hbm_pct_of_nominal_8tbs": round(100 * hbm / 8000.0, 2),
+        "roofline": {"bound": "hbm", "kernel": "index_topk", "achieved": round(achieved, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "peak_source": peaks["source"], "traffic": None,
+                     "launch_ms": round(topk_ms, 5), "algorithmic_bytes_per_launch": idx_bytes},
+        "kernel_ms": {"index_topk": round(topk_ms, 5), "sparse_decode": round(dec_ms, 5)},
+        "gpu_launches": QSADecodeStep.KERNELS_PER_STEP * K,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    return line
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        from workloads.qsa_inputs import WORKLOADS
+        w = WORKLOADS[args.workload]
+        per_step = 1
+        time_oracle(w, args.splits, per_step * max(1, args.warmup), seed=3000)
+        res = time_oracle(w, args.splits, per_step * args.steps, seed=3000)
+        line = {"metric": METRIC, "value": round(res["value"], 4), "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(1e3 * res["seconds"] / args.steps, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
+                "data": "synthetic", "config": {"workload": args.workload, "kv_splits": args.splits},
+                "cpu_baseline": {"value": round(res["value"], 4), "unit": UNIT, "cores": res["cores"],
+                                 "kind": "oracle",
+                                 "sample": f"{res['queries']} decode steps of {args.workload} (one "
+                                           f"request per step, cycling over {res['distinct']} drawn "
+                                           f"requests), NumPy oracle on 1 host core"},
+                "e2e": {"value": round(res["value"], 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    line = run_ours(args, rank, world, local_rank)
+    if rank == 0 and line is not None:
+        if not args.no_cpu_baseline:
+            from workloads.qsa_inputs import WORKLOADS
+            res = time_oracle(WORKLOADS[args.workload], args.splits, args.cpu_queries)
+            line["cpu_baseline"] = {"value": round(res["value"], 4), "unit": UNIT, "cores": res["cores"],
+                                    "kind": "oracle",
+                                    "sample": f"{res['queries']} decode steps of {args.workload} (one "
+                                              f"request each, cycling over {res['distinct']} drawn "
+                                              f"requests), NumPy oracle, {res['seconds']:.1f} s on "
+                                              f"1 host core"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,231 @@
+/*
+ * qsa.h — C ABI of the decode-time Qwen Sparse Attention (QSA) library
+ * (libqsa.so, hand-written CUDA kernels for sm_100a).
+ *
+ * The method (sources cited by page title and section):
+ *   - "Qwen 4 QSA 迎来解码上下文并行：深入解读 vLLM 针对 Qwen3.8-Flash-Next 的草稿 PR"
+ *     (orcarouter.ai), section "拉取请求实际改变了什么": a light indexer
+ *     compresses keys into micro-blocks at compression ratio 4, scores them
+ *     and keeps the best 512 blocks (about 2,048 token positions); the final
+ *     softmax and value aggregation still run on the uncompressed K and V.
+ *     Under decode context parallelism each rank reads its own slice of the
+ *     KV cache and the partial attention results are merged at the end; the
+ *     selector and its side caches are replicated and live in the same cache
+ *     group as the main KV cache.
+ *   - "PR #53896 完整报告" (prhub.com.cn), sections "执行摘要" / "实现拆解"
+ *     (weight-free top-k selector over a compressed-key cache; a circular
+ *     raw-key cache; MTP step 0 selects, later steps reuse the indices;
+ *     start-up check that the block size is divisible by the compress
+ *     ratio) and the QSAIndexer.forward excerpt under "关键源码片段"
+ *     (caches are updated and compressed before selection; the result is a
+ *     fixed-width row of request-relative indices padded with -1).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or keeps them.  Layouts are dense,
+ *     row-major (last index fastest) unless stated.
+ *   - Every call is asynchronous: it validates its host-side arguments,
+ *     enqueues kernels on `stream` and returns.  Arguments that can be
+ *     checked on the host are checked before anything is launched
+ *     (QSA_ERR_INVALID_ARG / QSA_ERR_UNSUPPORTED; nothing is launched then).
+ *   - Problems only visible on the device (a block-table entry out of range,
+ *     a context length that does not fit the block table, a malformed
+ *     selection row, a wait that ran out) are recorded in a per-device error
+ *     word and the offending access is skipped; read (and clear) it with
+ *     qsa_get_device_error().  No kernel traps.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).
+ */
+#ifndef QSA_H_
+#define QSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *qsa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1, /* a host-side argument is malformed            */
+  QSA_ERR_UNSUPPORTED = 2, /* a valid but unsupported shape or dtype        */
+  QSA_ERR_BOUNDS = 3,      /* device saw an out-of-range page / position    */
+  QSA_ERR_CUDA = 4,        /* a CUDA runtime call failed                    */
+  QSA_ERR_TIMEOUT = 5,     /* a bounded device wait ran out                 */
+  QSA_ERR_BAD_INPUT = 6    /* device saw malformed data (lengths, selection) */
+} qsa_status;
+
+typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype;
+
+/* Paged caches of one attention layer.  The main K/V cache, the compressed
+ * indexer-key cache and the block table form one cache group: the same
+ * block-table entry names the same physical page in all of them. */
+typedef struct {
+  int32_t num_pages;    /* physical pages in each cache                       */
+  int32_t page_size;    /* tokens per page P; multiple of 4 (compress ratio)  */
+  int32_t num_kv_heads; /* Hkv                                                */
+  int32_t head_dim;     /* D: 64 or 128                                       */
+  int32_t idx_dim;      /* indexer dim d: 32, 64 or 128                       */
+  int32_t kv_dtype;     /* qsa_dtype of k_cache / v_cache                     */
+  const void *k_cache;  /* [num_pages, P, Hkv, D] of kv_dtype                 */
+  const void *v_cache;  /* [num_pages, P, Hkv, D] of kv_dtype                 */
+  const float *k_scale; /* [num_pages, Hkv] dequant scale (FP8 only, else NULL) */
+  const float *v_scale; /* [num_pages, Hkv] dequant scale (FP8 only, else NULL) */
+  int16_t *kc;          /* [num_pages, P/4, d] compressed keys (sum of 4 int8 keys) */
+  int8_t *ring;         /* [ring_rows, 4, d] raw keys of the newest positions:
+                           slot p % 4 of row r holds request r's key at p     */
+  int32_t ring_rows;    /* rows of `ring` (>= batch of every call)            */
+  const int32_t *block_table; /* [B, max_pages_per_req] physical page of each
+                                 logical page; -1 = none                     */
+  int32_t max_pages_per_req;  /* row stride of block_table                    */
+} qsa_cache;
+
+/* Human-readable name of a status code (static string). */
+const char *qsa_status_string(int32_t status);
+
+/* Library ABI version (incremented on any incompatible change). */
+int32_t qsa_abi_version(void);
+
+/*
+ * qsa_compress_append — write new tokens' raw indexer keys and refresh the
+ * compressed key of every micro-block they touch.
+ *
+ * Passage: blog "拉取请求实际改变了什么" (keys compressed into micro-blocks
+ * at ratio 4); PR #53896 report, QSAIndexer.forward excerpt (token keys go
+ * to a circular raw-key cache, complete blocks are pooled into the
+ * compressed-key cache, before any selection).  Pooling is the plain
+ * integer sum: kc[b] = sum over tokens t in [4b, min(4b+4, end)) of k[t],
+ * so a partial tail block holds the sum of the tokens present.
+ *
+ *   B              requests in this call (<= cache->ring_rows)
+ *   pos0   [B]     int32, logical position of request r's first new token
+ *   cu_new [B+1]   int32, request r's new tokens are rows cu_new[r] ..
+ *                  cu_new[r+1]-1 of k_new (cu_new[0] = 0)
+ *   k_new  [N, d]  int8 raw indexer keys, N = cu_new[B]
+ *   max_new_per_req  host upper bound of cu_new[r+1]-cu_new[r] (sizes the
+ *                  launch; a request above it is an error on the device)
+ * Positions are appended in order: the raw keys of positions
+ * 4*floor(pos0/4) .. pos0-1 must have been appended by an earlier call (they
+ * are read back from ring row r).  A decode step passes T new tokens per
+ * request; a prefill passes whole chunks (complete blocks are pooled
+ * straight from k_new).  Errors: QSA_ERR_INVALID_ARG for null pointers,
+ * B < 0, B > ring_rows, page_size % 4 != 0 or an unsupported idx_dim.
+ */
+qsa_status qsa_compress_append(const qsa_cache *cache, int32_t B, const int32_t *pos0,
+                               const int32_t *cu_new, const int8_t *k_new,
+                               int32_t max_new_per_req, qsa_stream_t stream);
+
+/* Workspace bytes qsa_index_topk needs for B requests of at most
+ * max_blocks micro-blocks each. */
+size_t qsa_index_topk_workspace_bytes(int32_t B, int32_t max_blocks);
+
+/*
+ * qsa_index_topk — score every competing micro-block against the indexer
+ * query and keep the best `topk`.
+ *
+ * Passage: blog "拉取请求实际改变了什么" (score the micro-blocks, keep the
+ * best 512); PR #53896 report "执行摘要" (weight-free top-k selection) and
+ * QSAIndexer.forward excerpt (fixed-width int32 output padded with -1).
+ *
+ *   score[r][b] = sum_j q_idx[r][j] * kc_r[b][j]   (exact int32), b < n_r
+ *   n_r = n_sel[r] if n_sel != NULL else ceil(ctx_lens[r] / 4)
+ *   sel[r] = the topk blocks with the highest score (ties: lower block index
+ *            wins), listed in ascending block order, padded with -1
+ *
+ *   q_idx    [B, d] int8 indexer query (MTP: of query token 0)
+ *   ctx_lens [B] int32 tokens in each request's cache (>= 1)
+ *   n_sel    [B] int32 or NULL (MTP: floor((L - T) / 4) + 1)
+ *   max_blocks  host upper bound of n_r (row stride of the score buffer)
+ *   topk     1 .. 4096
+ *   sel      [B, topk] int32 output
+ *   scores   [B, max_blocks] int32 output of every score, or NULL
+ *   workspace  >= qsa_index_topk_workspace_bytes(B, max_blocks) bytes,
+ *            16-byte aligned, ZERO-FILLED before its first use; every
+ *            completed call leaves its counters zero again, so one
+ *            workspace serves any number of calls on one stream (calls
+ *            that overlap on the GPU need separate workspaces).
+ * The compressed-key pages are read through the block table.  Errors:
+ * QSA_ERR_INVALID_ARG (null pointer, topk or max_blocks out of range,
+ * workspace too small or misaligned, kc not 16-byte aligned).
+ */
+qsa_status qsa_index_topk(const qsa_cache *cache, int32_t B, const int8_t *q_idx,
+                          const int32_t *ctx_lens, const int32_t *n_sel, int32_t max_blocks,
+                          int32_t topk, int32_t *sel, int32_t *scores, void *workspace,
+                          size_t workspace_bytes, qsa_stream_t stream);
+
+/* Workspace bytes qsa_sparse_decode needs. */
+size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32_t Hkv,
+                                         int32_t D, int32_t topk, int32_t num_splits);
+
+/*
+ * qsa_sparse_decode — exact softmax attention over the selected tokens of
+ * the uncompressed paged K/V, split into KV partitions.
+ *
+ * Passage: blog "拉取请求实际改变了什么" (final softmax and value
+ * aggregation on the uncompressed K/V; each decode-context-parallel rank
+ * reads its own slice of the cache, results merged at the end); PR #53896
+ * report "实现拆解" (MTP step 0 selects, later steps reuse the indices).
+ *
+ * Query token t of request r sits at position p_t = L - T + t (p0 = L - T).
+ * It attends the set
+ *     { i in selected blocks : i <= p_t }  U  (p0, p_t]
+ * (the speculative tail is always visible, no token counted twice), with
+ * logits sm_scale * q . k_i and query head h reading kv head h / (Hq/Hkv).
+ * Split s owns logical pages [floor(s*NP/S), floor((s+1)*NP/S)),
+ * NP = ceil(L / P); it writes
+ *     lse_s = log sum_{i in split} exp(logit_i),
+ *     o_s   = sum_{i in split} exp(logit_i - lse_s) v_i,
+ * and an empty split writes o_s = 0, lse_s = -inf.  FP8 K/V values are
+ * code * scale[page][kv head].
+ *
+ *   q        [B, T, Hq, D] of q_dtype (QSA_F32 or QSA_BF16; BF16 for
+ *            BF16/FP8 caches, F32 for F32 caches)
+ *   sel      [B, topk] int32, ascending block indices padded with -1 (the
+ *            output of qsa_index_topk)
+ *   T        1 .. 4; (Hq/Hkv) * T <= 32; Hq % Hkv == 0
+ *   num_splits  1 .. 16
+ *   o_part   [S, B, T, Hq, D] float32 output
+ *   lse_part [S, B, T, Hq] float32 output (natural log)
+ *   workspace  >= qsa_sparse_decode_workspace_bytes(...), 16-byte aligned,
+ *            ZERO-FILLED before first use, left zeroed by every completed
+ *            call (same rule as qsa_index_topk).
+ * Errors: QSA_ERR_INVALID_ARG / QSA_ERR_UNSUPPORTED on the host; page or
+ * position violations -> QSA_ERR_BOUNDS on the device.
+ */
+qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
+                             const void *q, int32_t q_dtype, const int32_t *ctx_lens,
+                             const int32_t *sel, int32_t topk, float sm_scale,
+                             int32_t num_splits, float *o_part, float *lse_part,
+                             void *workspace, size_t workspace_bytes, qsa_stream_t stream);
+
+/*
+ * qsa_lse_merge — merge KV-partition partial results by log-sum-exp.
+ *
+ * Passage: blog "拉取请求实际改变了什么" (attention results from the ranks
+ * are merged at the end).
+ *   lse = log sum_s exp(lse_s),  o = sum_s exp(lse_s - lse) o_s;
+ *   when every lse_s is -inf: o = 0, lse = -inf.
+ *
+ *   o_part [S, rows, D], lse_part [S, rows] float32 (rows = B*T*Hq)
+ *   o [rows, D], lse [rows] float32 outputs (may not alias the inputs)
+ *   1 <= S <= 64, D % 4 == 0, all pointers 16-byte aligned.
+ */
+qsa_status qsa_lse_merge(int32_t num_splits, int64_t rows, int32_t D, const float *o_part,
+                         const float *lse_part, float *o, float *lse, qsa_stream_t stream);
+
+/*
+ * qsa_get_device_error — synchronise `stream`, then read and clear the
+ * current device's error word.  Returns QSA_OK when no kernel recorded a
+ * problem, else the first recorded code (QSA_ERR_BOUNDS, QSA_ERR_TIMEOUT,
+ * QSA_ERR_BAD_INPUT); *flags_out (if not NULL) receives every bit seen.
+ * The word is shared by all streams of the device.
+ */
+qsa_status qsa_get_device_error(qsa_stream_t stream, uint32_t *flags_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H_ */

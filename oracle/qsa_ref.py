@@ -89,6 +89,28 @@ def decode_values(arr: np.ndarray, kind: str) -> np.ndarray:
     raise ValueError(f"unknown value kind {kind!r}")
 
 
+class StoredRows:
+    """Logical K or V rows [L, Hkv, D] kept as stored (float32 values or
+    bf16 / e4m3 bit patterns) with an optional dequantisation scale per
+    (token, kv head) [L, Hkv].  Indexing decodes only the rows asked for and
+    returns exact float64 values (code * scale for FP8)."""
+
+    def __init__(self, stored: np.ndarray, kind: str, scale: np.ndarray | None = None):
+        self.stored, self.kind, self.scale = stored, kind, scale
+
+    @property
+    def shape(self):
+        return self.stored.shape
+
+    def __getitem__(self, idx):
+        vals = decode_values(self.stored[idx], self.kind)
+        if self.scale is None:
+            return vals
+        idx = idx if isinstance(idx, tuple) else (idx,)
+        sc = self.scale[idx[:2]].astype(np.float64)
+        return vals * sc[..., None] if vals.ndim > sc.ndim else vals * sc
+
+
 # ----------------------------------------------------------------------------
 # Indexer: compression, scoring, selection
 # ----------------------------------------------------------------------------
@@ -292,6 +314,7 @@ def decode_request(k_idx: np.ndarray, q_idx: np.ndarray, q: np.ndarray, K: np.nd
 
     k_idx int8 [L, d]; q_idx int8 [d] (indexer query of token 0);
     q float64 [T, Hq, D]; K, V float64 [L, Hkv, D] (already dequantised).
+    K and V may also be StoredRows views (decoded row by row on access).
     Returns kc, scores, sel, per-token o/lse (unsplit), o_part/lse_part per
     split and the merged o/lse.
     """

@@ -1,0 +1,192 @@
+"""Thin PyTorch binding of libqsa.so.
+
+The functions carry the names of the C entry points and do argument
+marshalling only: they check dtypes, shapes and contiguity on the host, pass
+raw device pointers and the current CUDA stream, and raise on a non-OK
+status.  Every step of the computation runs in the CUDA kernels; PyTorch only
+owns device memory and streams.  There is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+_KV_DTYPES = {torch.float32: _lib.QSA_F32, torch.bfloat16: _lib.QSA_BF16,
+              torch.float8_e4m3fn: _lib.QSA_FP8_E4M3}
+
+
+class QSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _lib.load()
+        super().__init__(f"{where}: {lib.qsa_status_string(status).decode()}")
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != _lib.QSA_OK:
+        raise QSAError(status, where)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to libqsa must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libqsa must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+@dataclass
+class QSACache:
+    """One attention layer's paged caches (a single cache group: the same
+    block-table entry names the same physical page in K, V and the
+    compressed-key cache)."""
+    k_cache: torch.Tensor               # [num_pages, P, Hkv, D] f32 / bf16 / fp8 e4m3
+    v_cache: torch.Tensor
+    kc: torch.Tensor                    # int16 [num_pages, P/4, d]
+    ring: torch.Tensor                  # int8 [ring_rows, 4, d]
+    block_table: torch.Tensor           # int32 [B, max_pages]
+    k_scale: torch.Tensor | None = None  # f32 [num_pages, Hkv] (fp8 only)
+    v_scale: torch.Tensor | None = None
+
+    @staticmethod
+    def allocate(k_cache, v_cache, block_table, idx_dim: int, ring_rows: int,
+                 k_scale=None, v_scale=None) -> "QSACache":
+        num_pages, P = k_cache.shape[0], k_cache.shape[1]
+        kc = torch.zeros((num_pages, P // 4, idx_dim), dtype=torch.int16, device=k_cache.device)
+        ring = torch.zeros((ring_rows, 4, idx_dim), dtype=torch.int8, device=k_cache.device)
+        return QSACache(k_cache, v_cache, kc, ring, block_table, k_scale, v_scale)
+
+    def struct(self) -> _lib.QsaCacheStruct:
+        k, v = self.k_cache, self.v_cache
+        if k.dtype not in _KV_DTYPES or v.dtype != k.dtype or k.shape != v.shape or k.dim() != 4:
+            raise TypeError("k_cache / v_cache must be [num_pages, P, Hkv, D] of one dtype "
+                            "(float32, bfloat16 or float8_e4m3fn)")
+        _need(self.kc, torch.int16, "kc")
+        _need(self.ring, torch.int8, "ring")
+        _need(self.block_table, torch.int32, "block_table")
+        num_pages, P, Hkv, D = k.shape
+        d = self.kc.shape[-1]
+        if self.kc.shape != (num_pages, P // 4, d) or self.ring.shape[1:] != (4, d):
+            raise ValueError("kc must be [num_pages, P/4, d] and ring [rows, 4, d]")
+        s = _lib.QsaCacheStruct()
+        s.num_pages, s.page_size, s.num_kv_heads, s.head_dim, s.idx_dim = num_pages, P, Hkv, D, d
+        s.kv_dtype = _KV_DTYPES[k.dtype]
+        s.k_cache, s.v_cache = _ptr(k), _ptr(v)
+        s.k_scale, s.v_scale = _ptr(self.k_scale), _ptr(self.v_scale)
+        s.kc, s.ring = _ptr(self.kc), _ptr(self.ring)
+        s.ring_rows = self.ring.shape[0]
+        s.block_table = _ptr(self.block_table)
+        s.max_pages_per_req = self.block_table.shape[1]
+        return s
+
+
+def qsa_compress_append(cache: QSACache, pos0: torch.Tensor, cu_new: torch.Tensor,
+                        k_new: torch.Tensor, max_new_per_req: int, stream=None) -> None:
+    _need(pos0, torch.int32, "pos0")
+    _need(cu_new, torch.int32, "cu_new")
+    _need(k_new, torch.int8, "k_new")
+    B = pos0.shape[0]
+    if cu_new.shape[0] != B + 1:
+        raise ValueError("cu_new must have B+1 entries")
+    s = cache.struct()
+    lib = _lib.load()
+    _check(lib.qsa_compress_append(ctypes.byref(s), B, _ptr(pos0), _ptr(cu_new), _ptr(k_new),
+                                   int(max_new_per_req), _stream(stream)), "qsa_compress_append")
+
+
+def qsa_index_topk_workspace_bytes(B: int, max_blocks: int) -> int:
+    return int(_lib.load().qsa_index_topk_workspace_bytes(B, max_blocks))
+
+
+def qsa_sparse_decode_workspace_bytes(B: int, T: int, Hq: int, Hkv: int, D: int, topk: int,
+                                      num_splits: int) -> int:
+    return int(_lib.load().qsa_sparse_decode_workspace_bytes(B, T, Hq, Hkv, D, topk, num_splits))
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """Zero-filled workspace (the counters at its start must begin at zero)."""
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def qsa_index_topk(cache: QSACache, q_idx: torch.Tensor, ctx_lens: torch.Tensor,
+                   n_sel: torch.Tensor | None, max_blocks: int, topk: int, sel: torch.Tensor,
+                   scores: torch.Tensor | None, workspace: torch.Tensor, stream=None) -> None:
+    _need(q_idx, torch.int8, "q_idx")
+    _need(ctx_lens, torch.int32, "ctx_lens")
+    _need(sel, torch.int32, "sel")
+    B = q_idx.shape[0]
+    if sel.shape != (B, topk):
+        raise ValueError("sel must be [B, topk]")
+    if n_sel is not None:
+        _need(n_sel, torch.int32, "n_sel")
+    if scores is not None:
+        _need(scores, torch.int32, "scores")
+        if scores.shape != (B, max_blocks):
+            raise ValueError("scores must be [B, max_blocks]")
+    s = cache.struct()
+    lib = _lib.load()
+    _check(lib.qsa_index_topk(ctypes.byref(s), B, _ptr(q_idx), _ptr(ctx_lens), _ptr(n_sel),
+                              int(max_blocks), int(topk), _ptr(sel), _ptr(scores),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)), "qsa_index_topk")
+
+
+def qsa_sparse_decode(cache: QSACache, q: torch.Tensor, ctx_lens: torch.Tensor,
+                      sel: torch.Tensor, sm_scale: float, num_splits: int,
+                      o_part: torch.Tensor, lse_part: torch.Tensor, workspace: torch.Tensor,
+                      stream=None) -> None:
+    B, T, Hq, D = q.shape
+    q_dt = {torch.float32: _lib.QSA_F32, torch.bfloat16: _lib.QSA_BF16}.get(q.dtype)
+    if q_dt is None:
+        raise TypeError("q must be float32 or bfloat16")
+    _need(ctx_lens, torch.int32, "ctx_lens")
+    _need(sel, torch.int32, "sel")
+    _need(o_part, torch.float32, "o_part")
+    _need(lse_part, torch.float32, "lse_part")
+    if o_part.shape != (num_splits, B, T, Hq, D) or lse_part.shape != (num_splits, B, T, Hq):
+        raise ValueError("o_part must be [S, B, T, Hq, D] and lse_part [S, B, T, Hq]")
+    s = cache.struct()
+    lib = _lib.load()
+    _check(lib.qsa_sparse_decode(ctypes.byref(s), B, T, Hq, _ptr(q), q_dt, _ptr(ctx_lens),
+                                 _ptr(sel), sel.shape[1], float(sm_scale), int(num_splits),
+                                 _ptr(o_part), _ptr(lse_part), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "qsa_sparse_decode")
+
+
+def qsa_lse_merge(o_part: torch.Tensor, lse_part: torch.Tensor, o: torch.Tensor,
+                  lse: torch.Tensor, stream=None) -> None:
+    for t, n in ((o_part, "o_part"), (lse_part, "lse_part"), (o, "o"), (lse, "lse")):
+        _need(t, torch.float32, n)
+    S, D = o_part.shape[0], o_part.shape[-1]
+    rows = lse_part[0].numel()
+    if o_part.numel() != S * rows * D or o.numel() != rows * D or lse.numel() != rows:
+        raise ValueError("shapes of o_part [S, rows, D], lse_part [S, rows], o [rows, D], lse [rows]")
+    lib = _lib.load()
+    _check(lib.qsa_lse_merge(S, rows, D, _ptr(o_part), _ptr(lse_part), _ptr(o), _ptr(lse),
+                             _stream(stream)), "qsa_lse_merge")
+
+
+def qsa_get_device_error(stream=None) -> tuple[int, int]:
+    """Synchronises the stream; returns (status, flag bits) and clears the
+    device error word."""
+    lib = _lib.load()
+    flags = ctypes.c_uint32(0)
+    st = lib.qsa_get_device_error(_stream(stream), ctypes.byref(flags))
+    return int(st), int(flags.value)

@@ -1,0 +1,376 @@
+// C-ABI entry points of libqsa.so (declared in include/qsa.h): host-side
+// validation, workspace layout and kernel launches.  Every step of the path
+// runs in the kernels included below; nothing here touches tensor data.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "qsa.h"
+#include "qsa_common.cuh"
+#include "compress_append.cuh"
+#include "index_topk.cuh"
+#include "sparse_decode.cuh"
+#include "lse_merge.cuh"
+
+namespace {
+
+using qsa::CacheDev;
+
+constexpr size_t kAlign = 256;
+// Both workspaces start with this many bytes of completion counters, which
+// must be zero before the first call and are left zero by every completed
+// call (the layout does not depend on the call's sizes).
+constexpr size_t kTicketBytes = 64 * 1024;
+constexpr int kMaxDevices = 64;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+qsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
+
+qsa_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+}
+
+qsa_status check_cache(const qsa_cache *c) {
+  if (!c) return QSA_ERR_INVALID_ARG;
+  if (c->page_size <= 0 || c->page_size % 4 != 0) return QSA_ERR_INVALID_ARG;
+  if (c->num_pages <= 0 || c->num_kv_heads <= 0 || c->max_pages_per_req <= 0)
+    return QSA_ERR_INVALID_ARG;
+  if (!c->block_table) return QSA_ERR_INVALID_ARG;
+  return QSA_OK;
+}
+
+CacheDev to_dev(const qsa_cache *c) {
+  CacheDev d;
+  d.num_pages = c->num_pages;
+  d.page_size = c->page_size;
+  d.num_kv_heads = c->num_kv_heads;
+  d.head_dim = c->head_dim;
+  d.idx_dim = c->idx_dim;
+  d.kv_dtype = c->kv_dtype;
+  d.k_cache = c->k_cache;
+  d.v_cache = c->v_cache;
+  d.k_scale = c->k_scale;
+  d.v_scale = c->v_scale;
+  d.kc = c->kc;
+  d.ring = c->ring;
+  d.ring_rows = c->ring_rows;
+  d.block_table = c->block_table;
+  d.max_pages_per_req = c->max_pages_per_req;
+  return d;
+}
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+
+int sm_count(int dev) {
+  static int cache[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+cudaError_t prepare_kernel(K kernel, size_t smem, bool *done_per_device) {
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxDevices && done_per_device[dev]) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done_per_device[dev] = true;
+  return e;
+}
+
+std::mutex g_mutex;
+
+// ------------------------------------------------------------------ topk --
+size_t topk_smem() { return sizeof(qsa::topk::Smem) + 128; }
+
+template <int DI>
+qsa_status launch_index_topk(const qsa::topk::Params &p, cudaStream_t stream) {
+  using namespace qsa::topk;
+  static bool done[kMaxDevices] = {false};
+  static int blocks_per_sm[kMaxDevices] = {0};
+  auto kernel = index_topk_kernel<DI>;
+  const size_t smem = topk_smem();
+  const int dev = current_device();
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (prepare_kernel(kernel, smem, done) != cudaSuccess) return QSA_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices && !blocks_per_sm[dev]) {
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, smem) != cudaSuccess)
+        return QSA_ERR_CUDA;
+      blocks_per_sm[dev] = n > 0 ? n : 1;
+    }
+  }
+  const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
+  const int grid = bps * sm_count(dev);
+  kernel<<<grid, kThreads, smem, stream>>>(p);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- decode --
+int decode_chunk_slots(int topk, int S) {
+  return (topk + 2 + qsa::dec::kChunkBlocks - 1) / qsa::dec::kChunkBlocks + S;
+}
+
+template <int D, int MT, bool FP8>
+qsa_status launch_decode_mma(const qsa::dec::Params &p, dim3 grid, cudaStream_t stream) {
+  static bool done[kMaxDevices] = {false};
+  auto kernel = qsa::dec::sparse_decode_mma_kernel<D, MT, FP8>;
+  const size_t smem = sizeof(qsa::dec::MmaSmem<D, MT, FP8>) + 128;
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (prepare_kernel(kernel, smem, done) != cudaSuccess) return QSA_ERR_CUDA;
+  }
+  kernel<<<grid, qsa::dec::kThreads, smem, stream>>>(p);
+  return launch_status();
+}
+
+template <int D>
+qsa_status launch_decode_f32(const qsa::dec::Params &p, dim3 grid, cudaStream_t stream) {
+  static bool done[kMaxDevices] = {false};
+  auto kernel = qsa::dec::sparse_decode_f32_kernel<D>;
+  const size_t smem = sizeof(qsa::dec::F32Smem<D>) + 128;
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (prepare_kernel(kernel, smem, done) != cudaSuccess) return QSA_ERR_CUDA;
+  }
+  kernel<<<grid, qsa::dec::kThreads, smem, stream>>>(p);
+  return launch_status();
+}
+
+template <int D>
+qsa_status dispatch_decode_d(const qsa::dec::Params &p, int kv_dtype, int MT, dim3 grid,
+                             cudaStream_t stream) {
+  if (kv_dtype == QSA_F32) return launch_decode_f32<D>(p, grid, stream);
+  const bool fp8 = kv_dtype == QSA_FP8_E4M3;
+  if (MT == 1) return fp8 ? launch_decode_mma<D, 1, true>(p, grid, stream)
+                          : launch_decode_mma<D, 1, false>(p, grid, stream);
+  return fp8 ? launch_decode_mma<D, 2, true>(p, grid, stream)
+             : launch_decode_mma<D, 2, false>(p, grid, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *qsa_status_string(int32_t status) {
+  switch (status) {
+    case QSA_OK: return "QSA_OK";
+    case QSA_ERR_INVALID_ARG: return "QSA_ERR_INVALID_ARG: malformed argument";
+    case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED: unsupported shape or dtype";
+    case QSA_ERR_BOUNDS: return "QSA_ERR_BOUNDS: page or position out of range";
+    case QSA_ERR_CUDA: return "QSA_ERR_CUDA: CUDA runtime error";
+    case QSA_ERR_TIMEOUT: return "QSA_ERR_TIMEOUT: a bounded device wait ran out";
+    case QSA_ERR_BAD_INPUT: return "QSA_ERR_BAD_INPUT: malformed lengths or selection";
+    default: return "unknown qsa_status";
+  }
+}
+
+int32_t qsa_abi_version(void) { return 1; }
+
+qsa_status qsa_compress_append(const qsa_cache *cache, int32_t B, const int32_t *pos0,
+                               const int32_t *cu_new, const int8_t *k_new,
+                               int32_t max_new_per_req, qsa_stream_t stream) {
+  qsa_status st = check_cache(cache);
+  if (st != QSA_OK) return st;
+  if (B < 0 || max_new_per_req < 0) return QSA_ERR_INVALID_ARG;
+  if (B == 0 || max_new_per_req == 0) return QSA_OK;
+  if (B > cache->ring_rows || B > 65535) return QSA_ERR_INVALID_ARG;
+  if (!pos0 || !cu_new || !k_new || !cache->kc || !cache->ring) return QSA_ERR_INVALID_ARG;
+  if (!aligned(k_new, 4) || !aligned(cache->kc, 8) || !aligned(cache->ring, 4))
+    return QSA_ERR_INVALID_ARG;
+  const long long max_blocks = (long long)max_new_per_req / 4 + 2;
+  const long long gx = (max_blocks + qsa::kAppendBlocksPerCta - 1) / qsa::kAppendBlocksPerCta;
+  if (gx > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)gx, (unsigned)B);
+  const CacheDev c = to_dev(cache);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (cache->idx_dim) {
+    case 32: qsa::compress_append_kernel<32><<<grid, qsa::kAppendThreads, 0, s>>>(c, B, pos0, cu_new, k_new, max_new_per_req); break;
+    case 64: qsa::compress_append_kernel<64><<<grid, qsa::kAppendThreads, 0, s>>>(c, B, pos0, cu_new, k_new, max_new_per_req); break;
+    case 128: qsa::compress_append_kernel<128><<<grid, qsa::kAppendThreads, 0, s>>>(c, B, pos0, cu_new, k_new, max_new_per_req); break;
+    default: return QSA_ERR_UNSUPPORTED;
+  }
+  return launch_status();
+}
+
+size_t qsa_index_topk_workspace_bytes(int32_t B, int32_t max_blocks) {
+  if (B < 0 || max_blocks < 0) return 0;
+  return kTicketBytes + align_up((size_t)B * (size_t)max_blocks * sizeof(int32_t));
+}
+
+qsa_status qsa_index_topk(const qsa_cache *cache, int32_t B, const int8_t *q_idx,
+                          const int32_t *ctx_lens, const int32_t *n_sel, int32_t max_blocks,
+                          int32_t topk, int32_t *sel, int32_t *scores, void *workspace,
+                          size_t workspace_bytes, qsa_stream_t stream) {
+  qsa_status st = check_cache(cache);
+  if (st != QSA_OK) return st;
+  if (B < 0) return QSA_ERR_INVALID_ARG;
+  if (topk < 1 || topk > qsa::topk::kMaxTopk) return QSA_ERR_INVALID_ARG;
+  if (max_blocks < 1 || max_blocks > (1 << 24)) return QSA_ERR_INVALID_ARG;
+  if (B == 0) return QSA_OK;
+  if ((size_t)B * sizeof(int32_t) > kTicketBytes) return QSA_ERR_UNSUPPORTED;
+  if (!q_idx || !ctx_lens || !sel || !workspace || !cache->kc) return QSA_ERR_INVALID_ARG;
+  if (cache->idx_dim != 32 && cache->idx_dim != 64 && cache->idx_dim != 128)
+    return QSA_ERR_UNSUPPORTED;
+  if (!aligned(cache->kc, 16) || !aligned(q_idx, 4) || !aligned(workspace, 16) ||
+      (scores && !aligned(scores, 4)))
+    return QSA_ERR_INVALID_ARG;
+  const size_t need = scores ? kTicketBytes : qsa_index_topk_workspace_bytes(B, max_blocks);
+  if (workspace_bytes < need) return QSA_ERR_INVALID_ARG;
+
+  qsa::topk::Params p;
+  p.c = to_dev(cache);
+  p.B = B;
+  p.q_idx = q_idx;
+  p.ctx_lens = ctx_lens;
+  p.n_sel = n_sel;
+  p.max_blocks = max_blocks;
+  p.topk = topk;
+  p.sel = sel;
+  p.tickets = static_cast<int32_t *>(workspace);
+  p.scores = scores ? scores
+                    : reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + kTicketBytes);
+  // Work units: about eight per resident CTA, each a whole number of stages.
+  const int stage_rows = qsa::topk::kStageBytes / (cache->idx_dim * 2);
+  const int dev = current_device();
+  const long long ctas = 2LL * sm_count(dev);
+  const long long total_rows = (long long)B * max_blocks;
+  long long ur = total_rows / (8 * ctas);
+  long long pow2 = stage_rows;
+  while (pow2 * 2 <= ur && pow2 < 8192) pow2 *= 2;
+  p.unit_rows = (int)pow2;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (cache->idx_dim) {
+    case 32: return launch_index_topk<32>(p, s);
+    case 64: return launch_index_topk<64>(p, s);
+    default: return launch_index_topk<128>(p, s);
+  }
+}
+
+size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32_t Hkv,
+                                         int32_t D, int32_t topk, int32_t num_splits) {
+  if (B < 0 || T < 1 || Hq < 1 || Hkv < 1 || D < 1 || topk < 1 || num_splits < 1) return 0;
+  const size_t M = (size_t)(Hq / Hkv) * T;
+  const size_t nch = decode_chunk_slots(topk, num_splits);
+  const size_t slots = (size_t)B * Hkv * nch;
+  return kTicketBytes + align_up(slots * M * D * sizeof(float)) + align_up(slots * M * sizeof(float));
+}
+
+qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
+                             const void *q, int32_t q_dtype, const int32_t *ctx_lens,
+                             const int32_t *sel, int32_t topk, float sm_scale,
+                             int32_t num_splits, float *o_part, float *lse_part,
+                             void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
+  qsa_status st = check_cache(cache);
+  if (st != QSA_OK) return st;
+  const int Hkv = cache->num_kv_heads;
+  const int D = cache->head_dim;
+  if (B < 0 || T < 1 || Hq < 1 || topk < 1 || topk > qsa::topk::kMaxTopk) return QSA_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > qsa::dec::kMaxSplits) return QSA_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return QSA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return QSA_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (T > qsa::dec::kMaxT || G * T > qsa::dec::kMaxRows) return QSA_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return QSA_ERR_UNSUPPORTED;
+  if (cache->kv_dtype == QSA_F32) {
+    if (q_dtype != QSA_F32) return QSA_ERR_UNSUPPORTED;
+  } else if (cache->kv_dtype == QSA_BF16 || cache->kv_dtype == QSA_FP8_E4M3) {
+    if (q_dtype != QSA_BF16) return QSA_ERR_UNSUPPORTED;
+  } else {
+    return QSA_ERR_UNSUPPORTED;
+  }
+  if (B == 0) return QSA_OK;
+  if (B > 65535 || Hkv > 65535) return QSA_ERR_UNSUPPORTED;
+  if ((size_t)B * Hkv * num_splits * sizeof(int32_t) > kTicketBytes) return QSA_ERR_UNSUPPORTED;
+  if (!q || !ctx_lens || !sel || !o_part || !lse_part || !workspace || !cache->k_cache ||
+      !cache->v_cache)
+    return QSA_ERR_INVALID_ARG;
+  if (cache->kv_dtype == QSA_FP8_E4M3 && (!cache->k_scale || !cache->v_scale))
+    return QSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(cache->k_cache, 16) || !aligned(cache->v_cache, 16) ||
+      !aligned(workspace, 16) || !aligned(o_part, 16))
+    return QSA_ERR_INVALID_ARG;
+  if (workspace_bytes < qsa_sparse_decode_workspace_bytes(B, T, Hq, Hkv, D, topk, num_splits))
+    return QSA_ERR_INVALID_ARG;
+
+  const int nch = decode_chunk_slots(topk, num_splits);
+  const int M = G * T;
+  qsa::dec::Params p;
+  p.c = to_dev(cache);
+  p.B = B;
+  p.T = T;
+  p.Hq = Hq;
+  p.G = G;
+  p.M = M;
+  p.q = q;
+  p.ctx_lens = ctx_lens;
+  p.sel = sel;
+  p.topk = topk;
+  p.scale_log2 = sm_scale * qsa::dec::kLog2e;
+  p.S = num_splits;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  p.tickets = reinterpret_cast<int32_t *>(ws);
+  const size_t slots = (size_t)B * Hkv * nch;
+  p.ws_o = reinterpret_cast<float *>(ws + kTicketBytes);
+  p.ws_lse = reinterpret_cast<float *>(ws + kTicketBytes + align_up(slots * M * D * sizeof(float)));
+  p.nch = nch;
+  const dim3 grid((unsigned)nch, (unsigned)Hkv, (unsigned)B);
+  const int MT = (M + 15) / 16;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (D == 64) return dispatch_decode_d<64>(p, cache->kv_dtype, MT, grid, s);
+  return dispatch_decode_d<128>(p, cache->kv_dtype, MT, grid, s);
+}
+
+qsa_status qsa_lse_merge(int32_t num_splits, int64_t rows, int32_t D, const float *o_part,
+                         const float *lse_part, float *o, float *lse, qsa_stream_t stream) {
+  if (num_splits < 1 || num_splits > qsa::kMergeMaxSplits || rows < 0 || D < 4 || D % 4 != 0)
+    return QSA_ERR_INVALID_ARG;
+  if (rows == 0) return QSA_OK;
+  if (!o_part || !lse_part || !o || !lse) return QSA_ERR_INVALID_ARG;
+  if (!aligned(o_part, 16) || !aligned(o, 16) || !aligned(lse_part, 4) || !aligned(lse, 4))
+    return QSA_ERR_INVALID_ARG;
+  const long long rows_per_cta = qsa::kMergeThreads / 32;
+  const long long grid = (rows + rows_per_cta - 1) / rows_per_cta;
+  if (grid > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  qsa::lse_merge_kernel<<<(unsigned)grid, qsa::kMergeThreads, 0,
+                          reinterpret_cast<cudaStream_t>(stream)>>>(num_splits, rows, D, o_part,
+                                                                    lse_part, o, lse);
+  return launch_status();
+}
+
+qsa_status qsa_get_device_error(qsa_stream_t stream, uint32_t *flags_out) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return QSA_ERR_CUDA;
+  uint32_t flags = 0;
+  if (cudaMemcpyFromSymbol(&flags, qsa::g_error_flags, sizeof(flags)) != cudaSuccess)
+    return QSA_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (flags && cudaMemcpyToSymbol(qsa::g_error_flags, &zero, sizeof(zero)) != cudaSuccess)
+    return QSA_ERR_CUDA;
+  if (flags_out) *flags_out = flags;
+  if (flags & qsa::kErrTimeout) return QSA_ERR_TIMEOUT;
+  if (flags & qsa::kErrBounds) return QSA_ERR_BOUNDS;
+  if (flags & qsa::kErrBadInput) return QSA_ERR_BAD_INPUT;
+  return QSA_OK;
+}
+
+}  // extern "C"

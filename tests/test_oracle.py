@@ -402,3 +402,21 @@ def test_depage_roundtrip():
     for i, p in enumerate(perm):
         kc_cache[p] = kc_logical[i * 2:(i + 1) * 2]
     assert np.array_equal(ref.depage_kc(kc_cache, perm, L, P), kc_logical[:math.ceil(L / 4)])
+
+
+def test_stored_rows_decode_matches_eager():
+    rng = np.random.default_rng(21)
+    L, Hkv, D = 11, 2, 4
+    bits = rng.integers(0, 256, size=(L, Hkv, D)).astype(np.uint8)
+    bits[bits == 0x7F] = 0x11
+    bits[bits == 0xFF] = 0x91
+    scale = rng.random((L, Hkv)) + 0.5
+    view = ref.StoredRows(bits, "e4m3", scale)
+    eager = ref.e4m3_bits_to_f64(bits) * scale[..., None]
+    toks = np.array([0, 3, 10])
+    assert np.array_equal(view[toks, 1, :], eager[toks, 1, :])
+    b16 = rng.integers(0, 1 << 16, size=(L, Hkv, D)).astype(np.uint16)
+    b16 = (b16 & 0x3FFF).astype(np.uint16)          # finite values only
+    v16 = ref.StoredRows(b16, "bf16")
+    assert np.array_equal(v16[toks, 0, :], ref.bf16_bits_to_f64(b16)[toks, 0, :])
+    assert v16.shape == (L, Hkv, D)

@@ -40,6 +40,7 @@ def test_planted_spans_win_selection():
         kc = ref.compress_keys(b.k_idx[a:e].numpy())
         s = ref.block_scores(b.q_idx[r].numpy(), kc)
         sel = ref.select_blocks(s, 512)
+        assert (b.planted_host[r] >= 0).all()
         assert set(b.planted_host[r].tolist()) <= set(sel.tolist())
         # planted attention keys: scaled logit near 8 for the first query head
         pg = request_pages(b, r)
@@ -62,3 +63,9 @@ def test_loguniform_lengths_in_range():
     from workloads.qsa_inputs import draw_ctx_lens
     L = draw_ctx_lens(WORKLOADS["mixed_fp8"], torch.Generator().manual_seed(0))
     assert L.shape == (256,) and int(L.min()) >= 4096 and int(L.max()) <= 1048576
+
+
+def test_short_requests_get_no_planted_spans():
+    b = make_batch(WORKLOADS["b32_32k"], "cpu", ctx_lens=[1, 20, 4096])
+    assert (b.planted_host[0] == -1).all() and (b.planted_host[1] == -1).all()
+    assert (b.planted_host[2] >= 0).all()

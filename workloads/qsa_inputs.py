@@ -152,12 +152,12 @@ def make_batch(w: QSAWorkload, device="cpu", seed: int | None = None,
 
     planted = None
     if w.planted:
-        planted = torch.zeros((B, w.planted), dtype=torch.int64)
+        # requests too short to hold the spans get none (row of -1)
+        planted = torch.full((B, w.planted), -1, dtype=torch.int64)
         for r in range(B):
             nfull = (int(L[r]) - w.T + 1) // RATIO        # complete blocks within [0, p0]
-            k = min(w.planted, nfull)
-            planted[r, :k] = torch.randperm(nfull, generator=meta)[:k]
-            planted[r, k:] = planted[r, 0]
+            if nfull >= w.planted:
+                planted[r] = torch.randperm(nfull, generator=meta)[:w.planted]
 
     dev_gen = torch.Generator(device=device).manual_seed(seed + 1)
     qdt = TORCH_DTYPES[w.q_dtype]
@@ -178,16 +178,19 @@ def make_batch(w: QSAWorkload, device="cpu", seed: int | None = None,
 
     # planted positions -> (physical page, offset) and the planted key values
     plant_pages = plant_offs = plant_rows = plant_k = None
-    if planted is not None:
+    if planted is not None and bool((planted >= 0).any()):
         toks = (planted[:, :, None] * RATIO + torch.arange(RATIO)[None, None, :]).reshape(B, -1)
         rows = torch.arange(B)[:, None].expand_as(toks)
-        plant_pages = table[rows, toks // P].to(torch.int64).reshape(-1)
-        plant_offs = (toks % P).reshape(-1)
-        plant_rows = rows.reshape(-1)
+        keep = (toks >= 0).reshape(-1)
+        toks_k = toks.reshape(-1)[keep]
+        rows_k = rows.reshape(-1)[keep]
+        plant_pages = table[rows_k, toks_k // P].to(torch.int64)
+        plant_offs = toks_k % P
+        plant_rows = rows_k
         qm = q[:, 0].float().reshape(B, w.Hkv, G, w.D).mean(dim=2) * alpha   # [B, Hkv, D]
-        plant_k = qm.cpu()[plant_rows]                                      # [B*8*4, Hkv, D]
+        plant_k = qm.cpu()[plant_rows]                                      # [n, Hkv, D]
         # indexer keys of planted tokens = the request's indexer query
-        glob = (cu[:-1][:, None] + toks).reshape(-1).to(device)
+        glob = (cu[:-1][rows_k] + toks_k).to(device)
         k_idx[glob] = q_idx[plant_rows.to(device)]
 
     if w.kv_dtype in ("f32", "bf16"):
@@ -196,7 +199,7 @@ def make_batch(w: QSAWorkload, device="cpu", seed: int | None = None,
             if dt == torch.float32 else _randn_bf16(shape, dev_gen, device)
         v_cache = torch.randn(shape, generator=dev_gen, device=device, dtype=torch.float32).to(dt) \
             if dt == torch.float32 else _randn_bf16(shape, dev_gen, device)
-        if planted is not None:
+        if plant_pages is not None:
             k_cache[plant_pages.to(device), plant_offs.to(device)] = plant_k.to(device=device, dtype=dt)
     else:
         k_cache = torch.empty(shape, device=device, dtype=torch.float8_e4m3fn)
@@ -209,7 +212,7 @@ def make_batch(w: QSAWorkload, device="cpu", seed: int | None = None,
             for cache, scale in ((k_cache, k_scale), (v_cache, v_scale)):
                 x = torch.randn((p1 - p0, P, w.Hkv, w.D), generator=dev_gen, device=device,
                                 dtype=torch.float32)
-                if cache is k_cache and planted is not None:
+                if cache is k_cache and plant_pages is not None:
                     sel = (plant_pages >= p0) & (plant_pages < p1)
                     if bool(sel.any()):
                         x[(plant_pages[sel] - p0).to(device), plant_offs[sel].to(device)] = \
