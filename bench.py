@@ -38,6 +38,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="b128_256k")
     ap.add_argument("--splits", type=int, default=2)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (profiling runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-queries", type=int, default=8,
@@ -262,6 +264,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = WORKLOADS[args.workload]
+    if args.batch is not None:
+        from dataclasses import replace
+        w = replace(w, batch=args.batch)
     S = args.splits
     batch = make_batch(w, dev, seed=w.seed + rank)
     B, T = w.batch, w.T

@@ -142,10 +142,10 @@ size_t qsa_index_topk_workspace_bytes(int32_t B, int32_t max_blocks);
  *   sel      [B, topk] int32 output
  *   scores   [B, max_blocks] int32 output of every score, or NULL
  *   workspace  >= qsa_index_topk_workspace_bytes(B, max_blocks) bytes,
- *            16-byte aligned, ZERO-FILLED before its first use; every
- *            completed call leaves its counters zero again, so one
- *            workspace serves any number of calls on one stream (calls
- *            that overlap on the GPU need separate workspaces).
+ *            16-byte aligned, any contents (it holds the scores when
+ *            `scores` is NULL); calls that overlap on the GPU need separate
+ *            workspaces.  Two kernels run: a scan that writes every score,
+ *            then a selection with one CTA per request.
  * The compressed-key pages are read through the block table.  Errors:
  * QSA_ERR_INVALID_ARG (null pointer, topk or max_blocks out of range,
  * workspace too small or misaligned, kc not 16-byte aligned).

@@ -8,50 +8,28 @@
 // index; kept blocks listed in ascending order.
 //
 // Design (B200): the scan is an HBM stream of int16 compressed keys
-// (256 B per block at d = 128).  A persistent grid (2 CTAs per SM) walks
-// fixed-size work units (request, run of blocks).  In each CTA one producer
-// thread streams 4 KiB stages of compressed-key rows from their pages into a
-// 16-stage shared-memory ring with cp.async.bulk (completion on mbarriers,
-// L2 evict-first); eight consumer warps turn each stage into 16..64 scores
-// with dp2a (int16 x int8 pairs) and a butterfly reduce-scatter, and write the
-// scores to an L2-resident buffer.  The CTA that finishes the last unit of a
-// request (atomic ticket) runs that request's selection while the other CTAs
-// keep streaming: a 4096-bin histogram of the high score bits finds the
-// threshold bin, the blocks above it are kept outright, the threshold bin's
-// blocks are gathered in shared memory and bitonic-sorted by (score desc,
-// index asc), and the kept indices are bitonic-sorted ascending.  A request
-// whose threshold bin overflows shared memory falls back to exact radix
-// passes over the score buffer.
+// (256 B per block at d = 128).  Persistent warps walk 8 KiB items (request,
+// run of rows), load them with 16-byte streaming loads (16 per lane in
+// flight), turn them into scores with dp2a (int16 x int8 pairs) and a
+// butterfly reduce-scatter, and write the scores to an L2-resident buffer.  A second kernel selects, one CTA per
+// request: a 4096-bin histogram of the high score bits finds the threshold
+// bin, the blocks above it are kept outright, the threshold bin's blocks are
+// gathered in shared memory and bitonic-sorted by (score desc, index asc),
+// and the kept indices are bitonic-sorted ascending.  A request whose
+// threshold bin overflows shared memory falls back to exact radix passes
+// over its scores.  (Selecting inside the scan kernel, in the CTA that
+// finished a request last, serialised the selections: that CTA fell behind
+// and kept finishing last.)
 #pragma once
 #include "qsa_common.cuh"
 
 namespace qsa {
 namespace topk {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;  // + one producer warp
-constexpr int kStageBytes = 4096;
-constexpr int kStages = 16;
 constexpr int kHistBins = 4096;  // first digit: bits [25:14] of score + 2^25
 constexpr int kCandCap = 2048;   // threshold-bin candidates kept in shared memory
 constexpr int kMaxTopk = 4096;
 constexpr int kScoreBias = 1 << 25;  // |score| <= 2^23 for d <= 128 and int8 inputs
-constexpr int kBarSelect = 1;        // named barrier of the consumer warps
-
-struct Smem {
-  alignas(128) uint8_t stage[kStages][kStageBytes];
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  int hist[kHistBins];  // also the kept-index list (kMaxTopk ints) after pass A
-  unsigned long long cand[kCandCap];
-  int warp_tot[kConsumerWarps];
-  int sel_req;     // request to select after this unit, or -1
-  int bin, above;  // threshold bin and count strictly above it
-  int nkeep, ncand;
-  int fb_key, fb_above, fb_idx;  // fallback path results
-  int abort_flag;                // a wait of this CTA gave up
-};
 
 struct Params {
   CacheDev c;
@@ -63,8 +41,6 @@ struct Params {
   int topk;
   int32_t *sel;
   int32_t *scores;   // [B, max_blocks]
-  int32_t *tickets;  // [B], zero between calls
-  int unit_rows;     // multiple of the rows of one stage
 };
 
 // Competing blocks of request r, validated the same way in every thread:
@@ -82,36 +58,6 @@ __device__ __forceinline__ int request_blocks(const Params &p, int r, bool repor
   return (int)n;
 }
 
-__device__ __forceinline__ int request_units(const Params &p, int n) {
-  return n > 0 ? ceil_div(n, p.unit_rows) : 1;
-}
-
-// Walks the persistent unit sequence u = blockIdx.x, += gridDim.x, mapping
-// each unit to (request, first row, rows).
-struct UnitWalker {
-  int r = 0, cum = 0, n = 0, units = 0;
-  bool report = false;
-  __device__ __forceinline__ void start(const Params &p, bool rep) {
-    report = rep;
-    r = 0;
-    cum = 0;
-    n = request_blocks(p, 0, report);
-    units = request_units(p, n);
-  }
-  // Advances to the request holding unit u; returns false past the end.
-  __device__ __forceinline__ bool seek(const Params &p, long long u) {
-    while (r < p.B && u >= (long long)cum + units) {
-      cum += units;
-      ++r;
-      if (r < p.B) {
-        n = request_blocks(p, r, report);
-        units = request_units(p, n);
-      }
-    }
-    return r < p.B;
-  }
-};
-
 // Order-preserving unsigned key of a score in [0, 2^26).  Valid inputs give
 // |score| <= 2^23; the clamp only keeps corrupt cache contents from indexing
 // outside the histogram.
@@ -121,11 +67,24 @@ __device__ __forceinline__ uint32_t score_key(int s) {
 }
 
 // ------------------------------------------------------------ selection --
+// One CTA of kSelThreads threads per request.  The request's scores (written
+// by the scan kernel, L2-resident) are read with 16-byte loads issued in
+// batches of kSelBatch per thread, so many loads are in flight at once.
+
+constexpr int kSelThreads = 512;
+constexpr int kSelBatch = 8;  // int4 loads in flight per thread
+
+struct SelSmem {
+  int hist[kHistBins];  // also the kept-index list (kMaxTopk ints) after pass A
+  unsigned long long cand[kCandCap];
+  int warp_tot[kSelThreads / 32];
+  int bin, above, nkeep, ncand, fb_key, fb_above, fb_idx;
+};
 
 __device__ __forceinline__ void bitonic_sort_u64(unsigned long long *a, int n_pow2, int tid) {
   for (int k = 2; k <= n_pow2; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < n_pow2; i += kConsumers) {
+      for (int i = tid; i < n_pow2; i += kSelThreads) {
         const int l = i ^ j;
         if (l > i) {
           const unsigned long long x = a[i], y = a[l];
@@ -136,7 +95,7 @@ __device__ __forceinline__ void bitonic_sort_u64(unsigned long long *a, int n_po
           }
         }
       }
-      named_bar_sync(kBarSelect, kConsumers);
+      __syncthreads();
     }
   }
 }
@@ -144,7 +103,7 @@ __device__ __forceinline__ void bitonic_sort_u64(unsigned long long *a, int n_po
 __device__ __forceinline__ void bitonic_sort_i32(int *a, int n_pow2, int tid) {
   for (int k = 2; k <= n_pow2; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < n_pow2; i += kConsumers) {
+      for (int i = tid; i < n_pow2; i += kSelThreads) {
         const int l = i ^ j;
         if (l > i) {
           const int x = a[i], y = a[l];
@@ -155,7 +114,7 @@ __device__ __forceinline__ void bitonic_sort_i32(int *a, int n_pow2, int tid) {
           }
         }
       }
-      named_bar_sync(kBarSelect, kConsumers);
+      __syncthreads();
     }
   }
 }
@@ -166,20 +125,45 @@ __device__ __forceinline__ int next_pow2(int x) {
   return p;
 }
 
-// Finds, in hist[0..nbins), the bin where the running count taken from the
-// top bin down (desc = true) or from bin 0 up first reaches `rank` (>= 1).
-// Writes the bin and the count strictly before it (in that order) to *bin and
-// *before.  Executed by all consumer threads; ends with a barrier.
-__device__ void find_rank_bin(const int *hist, int nbins, int rank, bool desc, int *bin,
-                              int *before, Smem &sm, int tid) {
-  const int per = nbins / kConsumers;  // nbins is a multiple of kConsumers
-  // thread t owns the t-th group of bins in the scan order
-  int local = 0;
-  for (int k = 0; k < per; ++k) {
-    const int b = desc ? (nbins - 1 - (tid * per + k)) : (tid * per + k);
-    local += hist[b];
+// Applies f(index, score) to every score of a row, reading it with batched
+// 16-byte loads from its first 16-byte boundary (rows are 4-byte aligned;
+// the row stride need not be a multiple of 4).
+template <typename F>
+__device__ __forceinline__ void for_each_score(const int32_t *sc, int n, int tid, F f) {
+  const int head = min(n, (int)(((16u - (uint32_t)(reinterpret_cast<uintptr_t>(sc) & 15u)) & 15u) >> 2));
+  if (tid < head) f(tid, __ldcg(sc + tid));
+  const int4 *v4 = reinterpret_cast<const int4 *>(sc + head);
+  const int nv = (n - head) >> 2;
+  for (int base = 0; base < nv; base += kSelThreads * kSelBatch) {
+    int4 v[kSelBatch];
+#pragma unroll
+    for (int j = 0; j < kSelBatch; ++j) {
+      const int i = base + j * kSelThreads + tid;
+      v[j] = (i < nv) ? __ldcg(v4 + i) : make_int4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < kSelBatch; ++j) {
+      const int i = base + j * kSelThreads + tid;
+      if (i < nv) {
+        const int e = head + 4 * i;
+        f(e, v[j].x);
+        f(e + 1, v[j].y);
+        f(e + 2, v[j].z);
+        f(e + 3, v[j].w);
+      }
+    }
   }
-  // exclusive scan over threads in scan order
+  for (int i = head + 4 * nv + tid; i < n; i += kSelThreads) f(i, __ldcg(sc + i));
+}
+
+// Finds, in hist[0..nbins), the bin where the running count taken from the
+// top bin down first reaches `rank` (>= 1); writes it and the count strictly
+// above it to sm.bin / sm.above.  Ends with a barrier.
+__device__ void find_rank_bin_desc(const int *hist, int rank, SelSmem &sm, int tid) {
+  constexpr int per = kHistBins / kSelThreads;
+  int local = 0;
+#pragma unroll
+  for (int k = 0; k < per; ++k) local += hist[kHistBins - 1 - (tid * per + k)];
   int incl = local;
   const int lane = tid & 31, w = tid >> 5;
 #pragma unroll
@@ -188,50 +172,46 @@ __device__ void find_rank_bin(const int *hist, int nbins, int rank, bool desc, i
     if (lane >= o) incl += v;
   }
   if (lane == 31) sm.warp_tot[w] = incl;
-  named_bar_sync(kBarSelect, kConsumers);
+  __syncthreads();
   int base = 0;
   for (int i = 0; i < w; ++i) base += sm.warp_tot[i];
   const int excl = base + incl - local;
   if (excl < rank && rank <= excl + local) {
     int cum = excl;
     for (int k = 0; k < per; ++k) {
-      const int b = desc ? (nbins - 1 - (tid * per + k)) : (tid * per + k);
+      const int b = kHistBins - 1 - (tid * per + k);
       if (cum + hist[b] >= rank) {
-        *bin = b;
-        *before = cum;
+        sm.bin = b;
+        sm.above = cum;
         break;
       }
       cum += hist[b];
     }
   }
-  named_bar_sync(kBarSelect, kConsumers);
+  __syncthreads();
 }
 
 // Exact fallback when the threshold bin does not fit in shared memory:
-// radix passes over the score buffer.  Establishes the exact threshold key,
-// then (on a tie at the threshold) the largest kept index among the tied
-// blocks, then gathers the kept set.
-__device__ void select_fallback(const int32_t *sc, int n, int K, Smem &sm, int tid) {
+// radix passes over the score row establish the exact threshold key, then
+// (on a tie at the threshold) the largest kept index among the tied blocks,
+// then the kept set is gathered.
+__device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, int tid) {
   int *hist = sm.hist;
-  const uint32_t b1 = (uint32_t)sm.bin;
-  // pass: bits [13:7] among keys with digit1 == b1; then bits [6:0]
-  uint32_t prefix = b1;  // key >> shift
+  uint32_t prefix = (uint32_t)sm.bin;  // key >> shift
   int above = sm.above;
   int shift = 14;
-  const int widths[2] = {7, 7};
   for (int pass = 0; pass < 2; ++pass) {
-    const int nb = 1 << widths[pass];
-    const int nshift = shift - widths[pass];
-    for (int i = tid; i < kHistBins; i += kConsumers) hist[i] = 0;
-    named_bar_sync(kBarSelect, kConsumers);
-    for (int i = tid; i < n; i += kConsumers) {
-      const uint32_t k = score_key(ld_cg_s32(sc + i));
-      if ((k >> shift) == prefix) atomicAdd(&hist[(k >> nshift) & (nb - 1)], 1);
-    }
-    named_bar_sync(kBarSelect, kConsumers);
+    const int nshift = shift - 7;
+    for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    for_each_score(sc, n, tid, [&](int, int s) {
+      const uint32_t k = score_key(s);
+      if ((k >> shift) == prefix) atomicAdd(&hist[(k >> nshift) & 127], 1);
+    });
+    __syncthreads();
     if (tid == 0) {
       int cum = above;
-      for (int b = nb - 1; b >= 0; --b) {
+      for (int b = 127; b >= 0; --b) {
         if (cum + hist[b] >= K) {
           sm.fb_key = b;
           sm.fb_above = cum;
@@ -240,35 +220,33 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, Smem &sm, int t
         cum += hist[b];
       }
     }
-    named_bar_sync(kBarSelect, kConsumers);
-    prefix = (prefix << widths[pass]) | (uint32_t)sm.fb_key;
+    __syncthreads();
+    prefix = (prefix << 7) | (uint32_t)sm.fb_key;
     above = sm.fb_above;
     shift = nshift;
   }
   const uint32_t tkey = prefix;  // exact threshold key
   const int need = K - above;    // tied blocks to keep, lowest indices first
-  // count ties; if some must be dropped, find the need-th smallest tied index
   if (tid == 0) sm.ncand = 0;
-  named_bar_sync(kBarSelect, kConsumers);
+  __syncthreads();
   int myties = 0;
-  for (int i = tid; i < n; i += kConsumers) myties += (score_key(ld_cg_s32(sc + i)) == tkey);
+  for_each_score(sc, n, tid, [&](int, int s) { myties += (score_key(s) == tkey); });
   atomicAdd(&sm.ncand, myties);
-  named_bar_sync(kBarSelect, kConsumers);
+  __syncthreads();
   int idx_limit = 0x7fffffff;
   if (sm.ncand > need) {
-    // radix select on the index (ascending), 3 passes of 8 bits over 24 bits
+    // radix select on the index (ascending): 3 passes of 8 bits (n <= 2^24)
     uint32_t ipre = 0;
     int before = 0;
     for (int pass = 0; pass < 3; ++pass) {
       const int sh = 16 - 8 * pass;
-      for (int i = tid; i < kHistBins; i += kConsumers) hist[i] = 0;
-      named_bar_sync(kBarSelect, kConsumers);
-      for (int i = tid; i < n; i += kConsumers) {
-        if (score_key(ld_cg_s32(sc + i)) != tkey) continue;
-        if (((uint32_t)i >> (sh + 8)) != ipre) continue;
-        atomicAdd(&hist[((uint32_t)i >> sh) & 255], 1);
-      }
-      named_bar_sync(kBarSelect, kConsumers);
+      for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+      __syncthreads();
+      for_each_score(sc, n, tid, [&](int i, int s) {
+        if (score_key(s) == tkey && ((uint32_t)i >> (sh + 8)) == ipre)
+          atomicAdd(&hist[((uint32_t)i >> sh) & 255], 1);
+      });
+      __syncthreads();
       if (tid == 0) {
         int cum = before;
         for (int b = 0; b < 256; ++b) {
@@ -280,270 +258,251 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, Smem &sm, int t
           cum += hist[b];
         }
       }
-      named_bar_sync(kBarSelect, kConsumers);
+      __syncthreads();
       ipre = (ipre << 8) | (uint32_t)sm.fb_idx;
       before = sm.fb_above;
     }
     idx_limit = (int)ipre;
   }
-  // gather the kept set
   int *keep = sm.hist;
   if (tid == 0) sm.nkeep = 0;
-  named_bar_sync(kBarSelect, kConsumers);
-  for (int i = tid; i < n; i += kConsumers) {
-    const uint32_t k = score_key(ld_cg_s32(sc + i));
+  __syncthreads();
+  for_each_score(sc, n, tid, [&](int i, int s) {
+    const uint32_t k = score_key(s);
     if (k > tkey || (k == tkey && i <= idx_limit)) {
       const int slot = atomicAdd(&sm.nkeep, 1);
       if (slot < kMaxTopk) keep[slot] = i;
     }
-  }
-  named_bar_sync(kBarSelect, kConsumers);
+  });
+  __syncthreads();
 }
 
-// Selection of request r by the kConsumers consumer threads.
-__device__ void select_request(const Params &p, int r, Smem &sm, int tid) {
-  const int n = request_blocks(p, r);
+// Selection kernel: grid = B, one request per CTA.
+__global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  SelSmem &sm = *reinterpret_cast<SelSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int r = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int n = request_blocks(p, r, tid == 0);
   const int K = p.topk;
   int32_t *out = p.sel + (long long)r * K;
   const int32_t *sc = p.scores + (long long)r * p.max_blocks;
   if (n <= K) {
-    for (int i = tid; i < K; i += kConsumers) out[i] = i < n ? i : -1;
+    for (int i = tid; i < K; i += kSelThreads) out[i] = i < n ? i : -1;
     return;
   }
   int *hist = sm.hist;
-  // pass A: histogram of the first digit
-  for (int i = tid; i < kHistBins; i += kConsumers) hist[i] = 0;
-  named_bar_sync(kBarSelect, kConsumers);
-  const int n4 = n & ~3;
-  for (int i = tid * 4; i < n4; i += kConsumers * 4) {
-    const int4 v = ld_cg_v4(sc + i);
-    atomicAdd(&hist[score_key(v.x) >> 14], 1);
-    atomicAdd(&hist[score_key(v.y) >> 14], 1);
-    atomicAdd(&hist[score_key(v.z) >> 14], 1);
-    atomicAdd(&hist[score_key(v.w) >> 14], 1);
-  }
-  for (int i = n4 + tid; i < n; i += kConsumers) atomicAdd(&hist[score_key(ld_cg_s32(sc + i)) >> 14], 1);
-  named_bar_sync(kBarSelect, kConsumers);
-  find_rank_bin(hist, kHistBins, K, true, &sm.bin, &sm.above, sm, tid);
+  // pass A: histogram of the first digit (bits [25:14] of the key)
+  for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+  __syncthreads();
+  for_each_score(sc, n, tid, [&](int, int s) { atomicAdd(&hist[score_key(s) >> 14], 1); });
+  __syncthreads();
+  find_rank_bin_desc(hist, K, sm, tid);
   const uint32_t b1 = (uint32_t)sm.bin;
-  // pass B: keep blocks above the bin; gather the bin's blocks
-  int *keep = sm.hist;  // histogram no longer needed
+  // pass B: keep the blocks above the threshold bin, gather the bin's blocks
+  int *keep = sm.hist;
   if (tid == 0) {
     sm.nkeep = 0;
     sm.ncand = 0;
   }
-  named_bar_sync(kBarSelect, kConsumers);
-  for (int i = tid; i < n; i += kConsumers) {
-    const uint32_t k = score_key(ld_cg_s32(sc + i));
+  __syncthreads();
+  for_each_score(sc, n, tid, [&](int i, int s) {
+    const uint32_t k = score_key(s);
     const uint32_t d1 = k >> 14;
     if (d1 > b1) {
       const int slot = atomicAdd(&sm.nkeep, 1);
       if (slot < kMaxTopk) keep[slot] = i;
     } else if (d1 == b1) {
       const int slot = atomicAdd(&sm.ncand, 1);
-      if (slot < kCandCap)
-        sm.cand[slot] = ((unsigned long long)(0xffffffffu - k) << 32) | (uint32_t)i;
+      if (slot < kCandCap) sm.cand[slot] = ((unsigned long long)(0xffffffffu - k) << 32) | (uint32_t)i;
     }
-  }
-  named_bar_sync(kBarSelect, kConsumers);
+  });
+  __syncthreads();
   const int above = sm.above;
   const int ncand = sm.ncand;
   if (ncand <= kCandCap) {
     const int np2 = next_pow2(ncand);
-    for (int i = ncand + tid; i < np2; i += kConsumers) sm.cand[i] = ~0ull;
-    named_bar_sync(kBarSelect, kConsumers);
+    for (int i = ncand + tid; i < np2; i += kSelThreads) sm.cand[i] = ~0ull;
+    __syncthreads();
     bitonic_sort_u64(sm.cand, np2, tid);
-    for (int j = tid; j < K - above; j += kConsumers)
+    for (int j = tid; j < K - above; j += kSelThreads)
       keep[above + j] = (int)(uint32_t)(sm.cand[j] & 0xffffffffu);
-    named_bar_sync(kBarSelect, kConsumers);
+    __syncthreads();
   } else {
     select_fallback(sc, n, K, sm, tid);
   }
-  // kept indices ascending
+  // kept indices in ascending order
   const int kp2 = next_pow2(K);
-  for (int i = K + tid; i < kp2; i += kConsumers) keep[i] = 0x7fffffff;
-  named_bar_sync(kBarSelect, kConsumers);
+  for (int i = K + tid; i < kp2; i += kSelThreads) keep[i] = 0x7fffffff;
+  __syncthreads();
   bitonic_sort_i32(keep, kp2, tid);
-  for (int i = tid; i < K; i += kConsumers) out[i] = keep[i];
+  for (int i = tid; i < K; i += kSelThreads) out[i] = keep[i];
 }
 
 // ------------------------------------------------------------- the scan --
+// Persistent warps stream the compressed keys straight into registers with
+// 16-byte loads: an item is 8 KiB of one request (16 loads per lane, all in
+// flight together), i.e. 4096/d rows; lane l reads dims 8*(l % LPR) .. +7 of
+// row (i * RPI + l / LPR) for load i.  Plain loads beat a shared-memory ring
+// fed by bulk copies here (measured on this GPU: ~7.0 vs ~3.9 TB/s on
+// randomly permuted 4 KiB pages).  The block-table entries of the next item
+// are fetched while the current one computes.
 
-// Butterfly reduce-scatter of 16 per-lane partial sums over groups of LPR
-// lanes (LPR = lanes that share one compressed-key row).
+constexpr int kScanThreads = 128;
+constexpr int kItemLoads = 16;  // 16-byte loads per lane per item (8 KiB per warp)
+
+__device__ __forceinline__ int pow2_log(int x) { return 31 - __clz(x); }
+
+// Reduce-scatter of 16 per-lane partial sums over groups of LPR lanes: after
+// log2(LPR) halving rounds lane l holds 16/LPR sums, value k being load index
+// ((l % LPR) << (4 - log2 LPR)) | k.
 template <int LPR>
 __device__ __forceinline__ void reduce_scatter16(int (&v)[16], int lane) {
   int n = 16;
 #pragma unroll
   for (int o = LPR / 2; o >= 1; o >>= 1) {
-    if (n > 1) {
-      const bool upper = (lane & o) != 0;
-      const int h = n / 2;
+    const bool upper = (lane & o) != 0;
+    const int h = n / 2;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (i < h) {
-          const int send = upper ? v[i] : v[i + h];
-          const int keepv = upper ? v[i + h] : v[i];
-          v[i] = keepv + __shfl_xor_sync(0xffffffffu, send, o);
-        }
+    for (int i = 0; i < 8; ++i) {
+      if (i < h) {
+        const int send = upper ? v[i] : v[i + h];
+        const int keepv = upper ? v[i + h] : v[i];
+        v[i] = keepv + __shfl_xor_sync(0xffffffffu, send, o);
       }
-      n = h;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
     }
+    n = h;
   }
 }
 
-template <int DI>
-__global__ void __launch_bounds__(kThreads, 2) index_topk_kernel(Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  constexpr int kRowBytes = DI * 2;
-  constexpr int kStageRows = kStageBytes / kRowBytes;  // 16 / 32 / 64
-  constexpr int kLPR = DI / 4;                         // lanes per row (8 B each)
-  constexpr int kRPI = 32 / kLPR;                      // rows per warp load
-  static_assert(kStageRows / kRPI == 16, "16 loads per lane per stage");
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int bpp = p.c.page_size / 4;
-
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
-    }
-    sm.sel_req = -1;
-    sm.abort_flag = 0;
-    fence_barrier_init();
+// Item walker: item it -> (request, first row).  Items are numbered request
+// after request; each warp visits it = warp_id, += total_warps.
+struct ItemWalker {
+  int r = 0, n = 0;
+  long long cum = 0, items = 0;
+  int rows_per_item = 0;
+  bool report = false;
+  __device__ __forceinline__ void start(const Params &p, int rpi, bool rep) {
+    rows_per_item = rpi;
+    report = rep;
+    r = 0;
+    cum = 0;
+    n = request_blocks(p, 0, report);
+    items = ceil_div_ll(n, rpi);
   }
-  __syncthreads();
-
-  const long long total_stride = gridDim.x;
-
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------ producer warp --
-    if (lane != 0) return;
-    const uint64_t pol = l2_policy_evict_first();
-    UnitWalker wk;
-    wk.start(p, blockIdx.x == 0);
-    long long g = 0;  // stage sequence number of this CTA
-    bool alive = true;
-    for (long long u = blockIdx.x; alive && wk.seek(p, u); u += total_stride) {
-      const int r = wk.r;
-      const long long row_begin = (u - wk.cum) * (long long)p.unit_rows;
-      const int rows = (int)max(0LL, min((long long)p.unit_rows, (long long)wk.n - row_begin));
-      const int nst = ceil_div(rows, kStageRows);
-      for (int st = 0; st < nst; ++st, ++g) {
-        const int slot = (int)(g % kStages);
-        const uint32_t par = (uint32_t)((g / kStages) & 1) ^ 1u;
-        if (!mbar_wait_abortable(&sm.empty[slot], par, &sm.abort_flag)) {
-          alive = false;
-          break;
-        }
-        const long long b0 = row_begin + (long long)st * kStageRows;
-        const int nrows = min(kStageRows, rows - st * kStageRows);
-        // bytes of the valid page segments of this stage
-        uint32_t bytes = 0;
-        for (int k = 0; k < nrows;) {
-          const long long b = b0 + k;
-          const int seg = min(nrows - k, bpp - (int)(b % bpp));
-          const long long lp = b / bpp;
-          if (lp < p.c.max_pages_per_req) {
-            const int pg = p.c.block_table[(long long)r * p.c.max_pages_per_req + lp];
-            if (pg >= 0 && pg < p.c.num_pages) bytes += seg * kRowBytes;
-          }
-          k += seg;
-        }
-        mbar_arrive_expect_tx(&sm.full[slot], bytes);
-        for (int k = 0; k < nrows;) {
-          const long long b = b0 + k;
-          const int seg = min(nrows - k, bpp - (int)(b % bpp));
-          const int pg = physical_page(p.c, r, b / bpp);
-          if (pg >= 0) {
-            const int16_t *src = p.c.kc + ((long long)pg * bpp + (b % bpp)) * DI;
-            bulk_g2s(&sm.stage[slot][k * kRowBytes], src, seg * kRowBytes, &sm.full[slot], pol);
-          }
-          k += seg;
-        }
+  __device__ __forceinline__ bool seek(const Params &p, long long it) {
+    while (r < p.B && it >= cum + items) {
+      cum += items;
+      ++r;
+      if (r < p.B) {
+        n = request_blocks(p, r, report);
+        items = ceil_div_ll(n, rows_per_item);
       }
     }
-    // Drain: every copy issued must land before the CTA may exit.
-    for (long long k = max(0LL, g - kStages); k < g; ++k)
-      if (!mbar_wait(&sm.full[k % kStages], (uint32_t)((k / kStages) & 1))) break;
-    return;
+    return r < p.B;
   }
+};
 
-  // ---------------------------------------------------- consumer warps --
-  UnitWalker wk;
-  wk.start(p, false);
-  long long g = 0;
+template <int DI>
+__global__ void __launch_bounds__(kScanThreads) index_scan_kernel(Params p) {
+  constexpr int kLPR = DI / 8;                    // lanes per row (16 B each)
+  constexpr int kRPI = 32 / kLPR;                 // rows per load instruction
+  constexpr int kRowsPerItem = kItemLoads * kRPI; // 4096 / DI
+  constexpr int kR = (kLPR == 16) ? 4 : (kLPR == 8) ? 3 : 2;
+  constexpr int kVals = 16 >> kR;
+  const int lane = threadIdx.x & 31;
+  const long long warp_id = ((long long)blockIdx.x * kScanThreads + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * kScanThreads) >> 5;
+  const int bpp = p.c.page_size / 4;
+  const int sub = lane % kLPR;                    // this lane's 8 dims: 8*sub .. 8*sub+7
+  const int row_in = lane / kLPR;
+
+  ItemWalker wk;
+  wk.start(p, kRowsPerItem, warp_id == 0 && lane == 0);
   int cur_r = -1;
-  uint32_t qword = 0;
-  for (long long u = blockIdx.x; wk.seek(p, u); u += total_stride) {
-    const int r = wk.r;
-    const long long row_begin = (u - wk.cum) * (long long)p.unit_rows;
-    const int rows = (int)max(0LL, min((long long)p.unit_rows, (long long)wk.n - row_begin));
-    const int nst = ceil_div(rows, kStageRows);
+  uint32_t q0 = 0, q1 = 0;
+
+  // block-table entries of an item: lane j holds logical page lp0 + j
+  // (rows and logical pages fit in 32 bits: n <= max_blocks <= 2^24)
+  auto fetch_pages = [&](int r, int row0, int &lp0_out) -> int {
+    const int lp0 = row0 / bpp;
+    lp0_out = lp0;
+    const int lp = lp0 + lane;
+    int v = -1;
+    if (lp < p.c.max_pages_per_req) {
+      v = p.c.block_table[(long long)r * p.c.max_pages_per_req + lp];
+      if (v >= p.c.num_pages) v = -1;
+    }
+    return v;
+  };
+
+  long long it = warp_id;
+  if (!wk.seek(p, it)) return;
+  int nr = wk.r;
+  int nrow0 = (int)(it - wk.cum) * kRowsPerItem;
+  int nlp0 = 0;
+  int npg = fetch_pages(nr, nrow0, nlp0);
+  while (true) {
+    const int r = nr;
+    const int row0 = nrow0;
+    const int lp0 = nlp0;
+    const int pg_lane = npg;
+    const int n = wk.n;
     if (r != cur_r) {
       cur_r = r;
-      qword = *reinterpret_cast<const uint32_t *>(p.q_idx + (long long)r * DI + (lane % kLPR) * 4);
+      const uint2 qq = *reinterpret_cast<const uint2 *>(p.q_idx + (long long)r * DI + sub * 8);
+      q0 = qq.x;
+      q1 = qq.y;
     }
-    int32_t *sc = p.scores + (long long)r * p.max_blocks;
-    for (int st = 0; st < nst; ++st, ++g) {
-      if ((int)(g % kConsumerWarps) != warp) continue;
-      const int slot = (int)(g % kStages);
-      const uint32_t par = (uint32_t)((g / kStages) & 1);
-      mbar_wait_abortable(&sm.full[slot], par, &sm.abort_flag);
-      const uint8_t *base = sm.stage[slot];
-      int acc[16];
+    // issue this item's loads
+    uint4 v[kItemLoads];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int row = i * kRPI + lane / kLPR;
-        const uint2 w = *reinterpret_cast<const uint2 *>(base + row * kRowBytes + (lane % kLPR) * 8);
-        int a = __dp2a_lo((int)w.x, (int)qword, 0);
-        acc[i] = __dp2a_hi((int)w.y, (int)qword, a);
+    for (int i = 0; i < kItemLoads; ++i) {
+      const int row = row0 + i * kRPI + row_in;
+      const int lp = row / bpp;
+      const int j = lp - lp0;
+      int pg = __shfl_sync(0xffffffffu, pg_lane, j & 31);
+      if (j >= 32) {  // item spans more than 32 pages (tiny pages): direct lookup
+        pg = (lp < p.c.max_pages_per_req) ? p.c.block_table[(long long)r * p.c.max_pages_per_req + lp] : -1;
+        if (pg >= p.c.num_pages) pg = -1;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[slot]);
-      reduce_scatter16<kLPR>(acc, lane);
-      const long long b0 = row_begin + (long long)st * kStageRows;
-      const int nrows = min(kStageRows, rows - st * kStageRows);
-      if constexpr (kLPR == 32) {
-        // lane pairs hold row (lane >> 1)
-        const int row = lane >> 1;
-        if ((lane & 1) == 0 && row < nrows) sc[b0 + row] = acc[0];
-      } else if constexpr (kLPR == 16) {
-        // lane holds i = lane & 15 of row group lane >> 4: row = i * 2 + (lane >> 4)
-        const int row = (lane & 15) * kRPI + (lane >> 4);
-        if (row < nrows) sc[b0 + row] = acc[0];
-      } else {
-        // kLPR == 8: lane holds i = ((lane & 7) << 1) | k, k = 0, 1
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int i = ((lane & 7) << 1) | k;
-          const int row = i * kRPI + (lane >> 3);
-          if (row < nrows) sc[b0 + row] = acc[k];
+      v[i] = make_uint4(0, 0, 0, 0);
+      if (row < n) {
+        if (pg >= 0) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(
+              p.c.kc + ((long long)pg * bpp + (row % bpp)) * DI + sub * 8);
+          v[i] = __ldcs(src);
+        } else if (lane == 0 || sub == 0) {
+          record_error(kErrBounds);
         }
       }
     }
-    // unit done: publish the scores, take a ticket
-    __threadfence();
-    named_bar_sync(kBarSelect, kConsumers);
-    if (tid == 0) {
-      const int t = atomicAdd(&p.tickets[r], 1);
-      sm.sel_req = (t == wk.units - 1) ? r : -1;
-      if (sm.sel_req >= 0) {
-        p.tickets[r] = 0;  // every unit of r has reported; reset for the next call
-        __threadfence();
-      }
+    // prefetch the next item's block-table entries
+    it += nwarps;
+    const bool more = wk.seek(p, it);
+    if (more) {
+      nr = wk.r;
+      nrow0 = (int)(it - wk.cum) * kRowsPerItem;
+      npg = fetch_pages(nr, nrow0, nlp0);
     }
-    named_bar_sync(kBarSelect, kConsumers);
-    const int sr = sm.sel_req;
-    if (sr >= 0) {
-      __threadfence();  // see every other CTA's published scores
-      select_request(p, sr, sm, tid);
-      named_bar_sync(kBarSelect, kConsumers);
+    // scores: dp2a of int16 pairs with int8 query pairs
+    int acc[16];
+#pragma unroll
+    for (int i = 0; i < kItemLoads; ++i) {
+      int a = __dp2a_lo((int)v[i].x, (int)q0, 0);
+      a = __dp2a_hi((int)v[i].y, (int)q0, a);
+      a = __dp2a_lo((int)v[i].z, (int)q1, a);
+      acc[i] = __dp2a_hi((int)v[i].w, (int)q1, a);
     }
+    reduce_scatter16<kLPR>(acc, lane);
+    int32_t *sc = p.scores + (long long)r * p.max_blocks;
+#pragma unroll
+    for (int k = 0; k < kVals; ++k) {
+      const int i = ((lane % kLPR) << (4 - kR)) | k;
+      const int row = row0 + i * kRPI + row_in;
+      if (row < n) sc[row] = acc[k];
+    }
+    if (!more) break;
   }
 }
 

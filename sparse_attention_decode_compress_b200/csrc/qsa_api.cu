@@ -30,8 +30,6 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-qsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
-
 qsa_status launch_status() {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
@@ -97,29 +95,33 @@ cudaError_t prepare_kernel(K kernel, size_t smem, bool *done_per_device) {
 std::mutex g_mutex;
 
 // ------------------------------------------------------------------ topk --
-size_t topk_smem() { return sizeof(qsa::topk::Smem) + 128; }
+size_t select_smem() { return sizeof(qsa::topk::SelSmem) + 128; }
 
+// Scan (persistent grid, scores to the buffer) then selection (one CTA per
+// request), back to back on the caller's stream.
 template <int DI>
 qsa_status launch_index_topk(const qsa::topk::Params &p, cudaStream_t stream) {
   using namespace qsa::topk;
-  static bool done[kMaxDevices] = {false};
+  static bool done_sel[kMaxDevices] = {false};
   static int blocks_per_sm[kMaxDevices] = {0};
-  auto kernel = index_topk_kernel<DI>;
-  const size_t smem = topk_smem();
+  auto kernel = index_scan_kernel<DI>;
   const int dev = current_device();
   {
     std::lock_guard<std::mutex> lk(g_mutex);
-    if (prepare_kernel(kernel, smem, done) != cudaSuccess) return QSA_ERR_CUDA;
+    if (prepare_kernel(select_kernel, select_smem(), done_sel) != cudaSuccess) return QSA_ERR_CUDA;
     if (dev >= 0 && dev < kMaxDevices && !blocks_per_sm[dev]) {
       int n = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, smem) != cudaSuccess)
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kScanThreads, 0) != cudaSuccess)
         return QSA_ERR_CUDA;
       blocks_per_sm[dev] = n > 0 ? n : 1;
     }
   }
   const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
   const int grid = bps * sm_count(dev);
-  kernel<<<grid, kThreads, smem, stream>>>(p);
+  kernel<<<grid, kScanThreads, 0, stream>>>(p);
+  qsa_status st = launch_status();
+  if (st != QSA_OK) return st;
+  select_kernel<<<p.B, kSelThreads, select_smem(), stream>>>(p);
   return launch_status();
 }
 
@@ -225,7 +227,7 @@ qsa_status qsa_index_topk(const qsa_cache *cache, int32_t B, const int8_t *q_idx
   if (topk < 1 || topk > qsa::topk::kMaxTopk) return QSA_ERR_INVALID_ARG;
   if (max_blocks < 1 || max_blocks > (1 << 24)) return QSA_ERR_INVALID_ARG;
   if (B == 0) return QSA_OK;
-  if ((size_t)B * sizeof(int32_t) > kTicketBytes) return QSA_ERR_UNSUPPORTED;
+  if (B > 0x7fffffff / 2) return QSA_ERR_UNSUPPORTED;
   if (!q_idx || !ctx_lens || !sel || !workspace || !cache->kc) return QSA_ERR_INVALID_ARG;
   if (cache->idx_dim != 32 && cache->idx_dim != 64 && cache->idx_dim != 128)
     return QSA_ERR_UNSUPPORTED;
@@ -244,18 +246,8 @@ qsa_status qsa_index_topk(const qsa_cache *cache, int32_t B, const int8_t *q_idx
   p.max_blocks = max_blocks;
   p.topk = topk;
   p.sel = sel;
-  p.tickets = static_cast<int32_t *>(workspace);
   p.scores = scores ? scores
                     : reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + kTicketBytes);
-  // Work units: about eight per resident CTA, each a whole number of stages.
-  const int stage_rows = qsa::topk::kStageBytes / (cache->idx_dim * 2);
-  const int dev = current_device();
-  const long long ctas = 2LL * sm_count(dev);
-  const long long total_rows = (long long)B * max_blocks;
-  long long ur = total_rows / (8 * ctas);
-  long long pow2 = stage_rows;
-  while (pow2 * 2 <= ur && pow2 < 8192) pow2 *= 2;
-  p.unit_rows = (int)pow2;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (cache->idx_dim) {
     case 32: return launch_index_topk<32>(p, s);

@@ -77,57 +77,73 @@ __device__ __forceinline__ int ext_block(const int32_t *sel_r, const Plan &pl, i
   return k < pl.nvalid ? sel_r[k] : pl.extra[k - pl.nvalid];
 }
 
+// Warp 0 reads the selection row once, coalesced (32 entries per load), and
+// counts, per split boundary, the selected blocks that start before it; the
+// list is ascending, so those counts are the boundaries in the extended list.
 __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl) {
   const int lane = threadIdx.x & 31;
   const int32_t *sel_r = p.sel + (long long)r * p.topk;
+  int L = p.ctx_lens[r];
+  if (L < p.T) {
+    if (lane == 0) record_error(kErrBadInput);
+    L = 0;
+  }
+  const int p0 = L - p.T;
+  const long long NP = ((long long)L + p.c.page_size - 1) / p.c.page_size;
+  // token boundary of split s (lane s holds boundary s, s = 1 .. S-1)
+  long long tb = 0;
+  if (lane >= 1 && lane < p.S) tb = min(((long long)lane * NP / p.S) * p.c.page_size, (long long)L);
+  int nvalid = 0, last = -1;
+  int below[kMaxSplits];  // below[s]: selected blocks starting before boundary s
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) below[s] = 0;
+  const int n_entries = (L > 0) ? p.topk : 0;
+  for (int base = 0; base < n_entries; base += 32 * 8) {
+    int v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int k = base + j * 32 + lane;
+      v[j] = (k < n_entries) ? sel_r[k] : -1;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool valid = v[j] >= 0;
+      nvalid += __popc(__ballot_sync(0xffffffffu, valid));
+      last = max(last, v[j]);
+#pragma unroll
+      for (int s = 1; s < kMaxSplits; ++s) {
+        if (s >= p.S) break;
+        const long long tbs = __shfl_sync(0xffffffffu, tb, s);
+        below[s] += __popc(__ballot_sync(0xffffffffu, valid && 4LL * v[j] < tbs));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
   if (lane == 0) {
-    int L = p.ctx_lens[r];
-    if (L < p.T) {
-      record_error(kErrBadInput);
-      L = 0;
-    }
     pl.L = L;
-    pl.p0 = L - p.T;
-    // selection rows are ascending and padded with -1: count the valid prefix
-    int lo = 0, hi = (L > 0) ? p.topk : 0;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (sel_r[mid] >= 0) lo = mid + 1; else hi = mid;
-    }
-    pl.nvalid = lo;
-    const int last = lo > 0 ? sel_r[lo - 1] : -1;
-    if (last >= 0 && 4LL * last > (long long)pl.p0) record_error(kErrBadInput);
+    pl.p0 = p0;
+    pl.nvalid = nvalid;
+    if (last >= 0 && 4LL * last > (long long)p0) record_error(kErrBadInput);
     int ne = 0;
     if (L > 0 && p.T > 1) {
-      const int bs = (pl.p0 + 1) >> 2, be = (L - 1) >> 2;
+      const int bs = (p0 + 1) >> 2, be = (L - 1) >> 2;
       for (int b = bs; b <= be && ne < 2; ++b)
         if (b > last) pl.extra[ne++] = b;
     }
     pl.n_extra = ne;
-    pl.nE = lo + ne;
-  }
-  __syncwarp();
-  // split boundaries in the extended list (lane s computes boundary s)
-  if (lane <= p.S) {
-    int eb;
-    if (lane == 0) {
-      eb = 0;
-    } else if (lane == p.S) {
-      eb = pl.nE;
-    } else {
-      const long long NP = ((long long)pl.L + p.c.page_size - 1) / p.c.page_size;
-      const long long tb = min(((long long)lane * NP / p.S) * p.c.page_size, (long long)pl.L);
-      int lo = 0, hi = pl.nE;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (4LL * ext_block(sel_r, pl, mid) < tb) lo = mid + 1; else hi = mid;
+    pl.nE = nvalid + ne;
+    pl.e_bound[0] = 0;
+    pl.e_bound[p.S] = pl.nE;
+#pragma unroll
+    for (int s = 1; s < kMaxSplits; ++s) {
+      if (s < p.S) {
+        const long long tbs = min(((long long)s * NP / p.S) * p.c.page_size, (long long)L);
+        int eb = below[s];
+        for (int x = 0; x < ne; ++x) eb += (4LL * pl.extra[x] < tbs);
+        pl.e_bound[s] = eb;
       }
-      eb = lo;
     }
-    pl.e_bound[lane] = eb;
-  }
-  __syncwarp();
-  if (lane == 0) {
     int cum = 0;
     pl.active = 0;
     for (int s = 0; s < p.S; ++s) {
@@ -171,9 +187,11 @@ __device__ void write_empty_splits(const Params &p, const Plan &pl, int r, int g
 // Writes this chunk's result (o_s [M][D] normalised, lse [M] natural log, in
 // shared memory) to the split outputs, merging the split's chunks when it is
 // the last of them to finish.
+// `wsm` is shared scratch of at least nch * M floats that the caller no
+// longer needs (it may alias o_s only beyond its first M * D floats).
 template <int D>
 __device__ void finish_chunk(const Params &p, const Plan &pl, int r, int g, const float *o_s,
-                             const float *lse_s, int *flag) {
+                             const float *lse_s, int *flag, float *wsm) {
   const int s = pl.split;
   if (pl.nchunks_split == 1) {
     for (int i = threadIdx.x; i < p.M * D; i += blockDim.x) {
@@ -200,19 +218,39 @@ __device__ void finish_chunk(const Params &p, const Plan &pl, int r, int g, cons
   __syncthreads();
   if (!*flag) return;
   __threadfence();
+  // merge the split's chunks: their lse into shared memory first (one batch
+  // of loads), then each output element reads its chunk partials with
+  // independent loads
   const long long slot0 = ((long long)r * Hkv + g) * p.nch + pl.first_chunk_of_split;
+  const int nc = pl.nchunks_split;
+  float *lse_c = wsm;  // [nc][M]
+  for (int i = threadIdx.x; i < nc * p.M; i += blockDim.x)
+    lse_c[i] = __ldcg(p.ws_lse + slot0 * p.M + i);
+  __syncthreads();
   for (int i = threadIdx.x; i < p.M * D; i += blockDim.x) {
     const int m = i / D, d = i % D;
     float mx = -INFINITY;
-    for (int c = 0; c < pl.nchunks_split; ++c)
-      mx = fmaxf(mx, ld_cg_f32(p.ws_lse + (slot0 + c) * p.M + m));
+    for (int c = 0; c < nc; ++c) mx = fmaxf(mx, lse_c[c * p.M + m]);
     float num = 0.f, den = 0.f;
     if (mx != -INFINITY) {
-      for (int c = 0; c < pl.nchunks_split; ++c) {
-        const float l = ld_cg_f32(p.ws_lse + (slot0 + c) * p.M + m);
+      int c = 0;
+      for (; c + 4 <= nc; c += 4) {
+        float ov[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) ov[u] = __ldcg(p.ws_o + ((slot0 + c + u) * p.M + m) * D + d);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float l = lse_c[(c + u) * p.M + m];
+          const float w = (l == -INFINITY) ? 0.f : __expf(l - mx);
+          den += w;
+          num += w * ov[u];
+        }
+      }
+      for (; c < nc; ++c) {
+        const float l = lse_c[c * p.M + m];
         const float w = (l == -INFINITY) ? 0.f : __expf(l - mx);
         den += w;
-        num += w * ld_cg_f32(p.ws_o + ((slot0 + c) * p.M + m) * D + d);
+        num += w * __ldcg(p.ws_o + ((slot0 + c) * p.M + m) * D + d);
       }
     }
     p.o_part[out_row(p, s, r, g, m) * D + d] = den > 0.f ? num / den : 0.f;
@@ -286,6 +324,12 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// 2^x with the SFU approximation (relative error about 2^-22); -inf -> 0.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -487,13 +531,13 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_mma_kernel(Params p) {
         const float m_old = mrow[mt][hr];
         const float m_new = fmaxf(m_old, mx);
         const float base = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = exp2f(m_old - base);  // m_old = -inf -> 0
+        const float alpha = ex2(m_old - base);  // m_old = -inf -> 0
         mrow[mt][hr] = m_new;
         float psum = 0.f;
         float pv[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float pj = exp2f(x[j] - base);
+          const float pj = ex2(x[j] - base);
           psum += pj;
           const int slot = st * kStageTokens + tok0 + (j >> 1) * 8 + 2 * cq + (j & 1);
           pv[j] = FP8 ? pj * sm.tm.vs[slot] : pj;
@@ -594,7 +638,7 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_mma_kernel(Params p) {
     if (d == 0) sm.lse[m] = den > 0.f ? (mx + __log2f(den)) * kLn2 : -INFINITY;
   }
   __syncthreads();
-  finish_chunk<D>(p, pl, r, g, ow, sm.lse, &sm.flag);
+  finish_chunk<D>(p, pl, r, g, ow, sm.lse, &sm.flag, ow + p.M * D);
 }
 
 // ------------------------------------------------------- fp32 K/V path --
@@ -606,6 +650,7 @@ struct F32Smem {
   Plan pl;
   float o[kMaxRows * D];
   float lse[kMaxRows];
+  float scratch[kMaxRows * (4096 / kChunkBlocks + 2 + kMaxSplits)];
   int flag;
 };
 
@@ -657,7 +702,7 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_f32_kernel(Params p) {
     if (lane == 0) sm.lse[m] = l > 0.f ? (mx + __log2f(l)) * kLn2 : -INFINITY;
   }
   __syncthreads();
-  finish_chunk<D>(p, pl, r, g, sm.o, sm.lse, &sm.flag);
+  finish_chunk<D>(p, pl, r, g, sm.o, sm.lse, &sm.flag, sm.scratch);
 }
 
 }  // namespace dec

@@ -40,5 +40,5 @@ class QSADecodeStep:
         qsa_lse_merge(self.o_part, self.lse_part, self.o, self.lse, stream)
         return self.o, self.lse
 
-    # number of kernels one call launches (one per step of the path)
-    KERNELS_PER_STEP = 4
+    # kernels one call launches: append, scan + select, decode, merge
+    KERNELS_PER_STEP = 5
