@@ -454,12 +454,14 @@ __global__ void __launch_bounds__(kScanThreads) index_scan_kernel(Params p) {
       q0 = qq.x;
       q1 = qq.y;
     }
-    // issue this item's loads
+    // issue this item's loads; the lane's row advances by kRPI per load, so
+    // its (logical page, row in page) pair is stepped instead of divided
     uint4 v[kItemLoads];
+    int lp = (row0 + row_in) / bpp;
+    int off = (row0 + row_in) - lp * bpp;
 #pragma unroll
     for (int i = 0; i < kItemLoads; ++i) {
       const int row = row0 + i * kRPI + row_in;
-      const int lp = row / bpp;
       const int j = lp - lp0;
       int pg = __shfl_sync(0xffffffffu, pg_lane, j & 31);
       if (j >= 32) {  // item spans more than 32 pages (tiny pages): direct lookup
@@ -470,11 +472,16 @@ __global__ void __launch_bounds__(kScanThreads) index_scan_kernel(Params p) {
       if (row < n) {
         if (pg >= 0) {
           const uint4 *src = reinterpret_cast<const uint4 *>(
-              p.c.kc + ((long long)pg * bpp + (row % bpp)) * DI + sub * 8);
+              p.c.kc + ((long long)pg * bpp + off) * DI + sub * 8);
           v[i] = __ldcs(src);
         } else if (lane == 0 || sub == 0) {
           record_error(kErrBounds);
         }
+      }
+      off += kRPI;
+      while (off >= bpp) {
+        off -= bpp;
+        ++lp;
       }
     }
     // prefetch the next item's block-table entries

@@ -13,6 +13,7 @@
 #include "compress_append.cuh"
 #include "index_topk.cuh"
 #include "sparse_decode.cuh"
+#include "sparse_decode_warp.cuh"
 #include "lse_merge.cuh"
 
 namespace {
@@ -130,16 +131,36 @@ int decode_chunk_slots(int topk, int S) {
   return (topk + 2 + qsa::dec::kChunkBlocks - 1) / qsa::dec::kChunkBlocks + S;
 }
 
-template <int D, int MT, bool FP8>
-qsa_status launch_decode_mma(const qsa::dec::Params &p, dim3 grid, cudaStream_t stream) {
+// Worker warps per SM and ring depth of the tensor-core decode kernel: as
+// many warps as registers allow (query-row tiles NT set the accumulator
+// size), then as deep a ring as shared memory allows.
+template <int D, int NT, bool FP8>
+struct DecodeShape {
+  static constexpr int NW = (!FP8 && NT <= 2) ? 12 : 8;
+  static constexpr int NS = (!FP8 && NT <= 2) ? 2 : (FP8 ? 4 : 3);
+};
+
+template <int D, int NT, bool FP8>
+qsa_status launch_decode_warp(const qsa::dec::Params &p, cudaStream_t stream) {
+  constexpr int NW = DecodeShape<D, NT, FP8>::NW;
+  constexpr int NS = DecodeShape<D, NT, FP8>::NS;
   static bool done[kMaxDevices] = {false};
-  auto kernel = qsa::dec::sparse_decode_mma_kernel<D, MT, FP8>;
-  const size_t smem = sizeof(qsa::dec::MmaSmem<D, MT, FP8>) + 128;
+  static int blocks_per_sm[kMaxDevices] = {0};
+  auto kernel = qsa::dec::sparse_decode_warp_kernel<D, NT, FP8, NW, NS>;
+  const size_t smem = sizeof(qsa::dec::WarpSmem<D, FP8, NW, NS>) + 128;
+  const int dev = current_device();
   {
     std::lock_guard<std::mutex> lk(g_mutex);
     if (prepare_kernel(kernel, smem, done) != cudaSuccess) return QSA_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices && !blocks_per_sm[dev]) {
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, NW * 32, smem) != cudaSuccess)
+        return QSA_ERR_CUDA;
+      blocks_per_sm[dev] = n > 0 ? n : 1;
+    }
   }
-  kernel<<<grid, qsa::dec::kThreads, smem, stream>>>(p);
+  const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
+  kernel<<<bps * sm_count(dev), NW * 32, smem, stream>>>(p);
   return launch_status();
 }
 
@@ -156,15 +177,23 @@ qsa_status launch_decode_f32(const qsa::dec::Params &p, dim3 grid, cudaStream_t 
   return launch_status();
 }
 
+template <int D, bool FP8>
+qsa_status dispatch_decode_nt(const qsa::dec::Params &p, int NT, cudaStream_t stream) {
+  switch (NT) {
+    case 1: return launch_decode_warp<D, 1, FP8>(p, stream);
+    case 2: return launch_decode_warp<D, 2, FP8>(p, stream);
+    case 3: return launch_decode_warp<D, 3, FP8>(p, stream);
+    default: return launch_decode_warp<D, 4, FP8>(p, stream);
+  }
+}
+
 template <int D>
-qsa_status dispatch_decode_d(const qsa::dec::Params &p, int kv_dtype, int MT, dim3 grid,
+qsa_status dispatch_decode_d(const qsa::dec::Params &p, int kv_dtype, dim3 grid,
                              cudaStream_t stream) {
   if (kv_dtype == QSA_F32) return launch_decode_f32<D>(p, grid, stream);
-  const bool fp8 = kv_dtype == QSA_FP8_E4M3;
-  if (MT == 1) return fp8 ? launch_decode_mma<D, 1, true>(p, grid, stream)
-                          : launch_decode_mma<D, 1, false>(p, grid, stream);
-  return fp8 ? launch_decode_mma<D, 2, true>(p, grid, stream)
-             : launch_decode_mma<D, 2, false>(p, grid, stream);
+  const int NT = (p.M + 7) / 8;  // query rows on the N side, tiles of 8
+  if (kv_dtype == QSA_FP8_E4M3) return dispatch_decode_nt<D, true>(p, NT, stream);
+  return dispatch_decode_nt<D, false>(p, NT, stream);
 }
 
 }  // namespace
@@ -290,7 +319,9 @@ qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32
   }
   if (B == 0) return QSA_OK;
   if (B > 65535 || Hkv > 65535) return QSA_ERR_UNSUPPORTED;
-  if ((size_t)B * Hkv * num_splits * sizeof(int32_t) > kTicketBytes) return QSA_ERR_UNSUPPORTED;
+  if ((size_t)B * Hkv * num_splits * sizeof(int32_t) >
+      kTicketBytes - qsa::dec::kCounterInts * sizeof(int32_t))
+    return QSA_ERR_UNSUPPORTED;
   if (!q || !ctx_lens || !sel || !o_part || !lse_part || !workspace || !cache->k_cache ||
       !cache->v_cache)
     return QSA_ERR_INVALID_ARG;
@@ -320,16 +351,16 @@ qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32
   p.o_part = o_part;
   p.lse_part = lse_part;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  p.tickets = reinterpret_cast<int32_t *>(ws);
+  p.counters = reinterpret_cast<int32_t *>(ws);
+  p.tickets = p.counters + qsa::dec::kCounterInts;
   const size_t slots = (size_t)B * Hkv * nch;
   p.ws_o = reinterpret_cast<float *>(ws + kTicketBytes);
   p.ws_lse = reinterpret_cast<float *>(ws + kTicketBytes + align_up(slots * M * D * sizeof(float)));
   p.nch = nch;
   const dim3 grid((unsigned)nch, (unsigned)Hkv, (unsigned)B);
-  const int MT = (M + 15) / 16;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (D == 64) return dispatch_decode_d<64>(p, cache->kv_dtype, MT, grid, s);
-  return dispatch_decode_d<128>(p, cache->kv_dtype, MT, grid, s);
+  if (D == 64) return dispatch_decode_d<64>(p, cache->kv_dtype, grid, s);
+  return dispatch_decode_d<128>(p, cache->kv_dtype, grid, s);
 }
 
 qsa_status qsa_lse_merge(int32_t num_splits, int64_t rows, int32_t D, const float *o_part,

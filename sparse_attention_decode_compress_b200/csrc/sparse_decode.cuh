@@ -8,24 +8,19 @@
 // 什么).  MTP: the selection of query token 0 is reused by the speculative
 // tokens (PR #53896 完整报告, 实现拆解), which also see the speculative tail.
 //
-// Work decomposition: one CTA per (request r, kv head g, chunk).  The
-// "extended selection" of r is the sorted selection row followed by the
-// speculative-tail blocks that are not selected; split s owns the entries
-// whose block lies in its page slice (a contiguous range, since the list is
-// sorted), cut into chunks of 64 micro-blocks (256 tokens).  Each CTA gathers
-// its chunk's K/V rows for head g (cp.async, 16 B per thread, XOR-swizzled
-// rows), 64 tokens per stage, double-buffered; four warps each take 16 tokens
-// of a stage and run an online softmax:
-//   S = Q K^T  with mma.sync m16n8k16 bf16 -> fp32 (Q rows = the G query
-//              heads of g times the T query tokens, padded to 16 or 32),
-//   P = exp2(S*scale*log2e - m) kept in fp32 and fed to the P.V product as a
-//       bf16 hi + bf16 lo pair (two MMAs), so P carries ~16 significant bits.
-// The four warps' states are merged in shared memory into the chunk's
-// (o, lse).  A split with one chunk writes o_part/lse_part directly; a split
-// with several chunks stages them in the workspace and the CTA that finishes
-// last (atomic ticket) merges them by log-sum-exp.  FP8 E4M3 rows are
-// converted to bf16 in shared memory (exact); the per-(page, head) K scale
-// multiplies the logits and the V scale multiplies P.
+// Work decomposition (shared by both kernels): work items are (request r,
+// kv head g, chunk).  The "extended selection" of r is the sorted selection
+// row followed by the speculative-tail blocks that are not selected; split s
+// owns the entries whose block lies in its page slice (a contiguous range,
+// since the list is sorted), cut into chunks of 64 micro-blocks (256 tokens).
+// A split with one chunk writes o_part/lse_part directly; a split with
+// several chunks stages them in the workspace and the chunk that finishes
+// last (atomic ticket) merges them by log-sum-exp.
+//
+// This file holds the split/chunk plan, the output helpers and the plain
+// CUDA-core kernel for fp32 caches (one CTA per item, online softmax per
+// query row); the tensor-core kernel for bf16 / fp8 caches is in
+// sparse_decode_warp.cuh.
 #pragma once
 #include "qsa_common.cuh"
 
@@ -57,8 +52,9 @@ struct Params {
   float *lse_part;  // [S, B, T, Hq]
   float *ws_o;      // [B, Hkv, nch, M, D]
   float *ws_lse;    // [B, Hkv, nch, M]
-  int32_t *tickets; // [B, Hkv, S]
-  int nch;          // chunk slots per (r, g)
+  int32_t *tickets;  // [B, Hkv, S]
+  int32_t *counters; // work counters of the persistent kernel (zero between calls)
+  int nch;           // chunk slots per (r, g)
 };
 
 // Per-CTA plan, computed by warp 0.
@@ -341,304 +337,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 template <int D>
 __device__ __forceinline__ int swz(int row, int ch) {
   return row * (D * 2) + ((ch ^ (row & 7)) << 4);
-}
-
-template <int D, int MT, bool FP8>
-struct MmaSmem {
-  alignas(128) uint8_t kv[2][2][kStageTokens * D * 2];  // [buffer][K=0 / V=1] swizzled bf16
-  alignas(128) uint8_t raw[2][2][FP8 ? kStageTokens * D : 16];  // fp8 landing rows
-  alignas(128) uint8_t q[MT * 16 * D * 2];              // swizzled bf16 Q rows
-  TokMeta tm;
-  Plan pl;
-  float wm[kWarps][MT * 16];
-  float wl[kWarps][MT * 16];
-  float lse[kMaxRows];
-  int flag;
-};
-
-// Issues the cp.async loads of stage `st` of the chunk into buffer `buf`.
-template <int D, bool FP8>
-__device__ __forceinline__ void load_stage(const Params &p, uint8_t *kdst, uint8_t *vdst,
-                                           const TokMeta &tm, int st) {
-  constexpr int kElemBytes = FP8 ? 1 : 2;
-  constexpr int kRowBytes = D * kElemBytes;
-  constexpr int kChunksPerRow = kRowBytes / 16;
-  constexpr int kItems = kStageTokens * kChunksPerRow;
-  const uint8_t *kbase = static_cast<const uint8_t *>(p.c.k_cache);
-  const uint8_t *vbase = static_cast<const uint8_t *>(p.c.v_cache);
-  for (int it = threadIdx.x; it < 2 * kItems; it += kThreads) {
-    const int kv = it / kItems;
-    const int rem = it % kItems;
-    const int row = rem / kChunksPerRow, ch = rem % kChunksPerRow;
-    const long long off = tm.off[st * kStageTokens + row];
-    uint8_t *dst = (kv ? vdst : kdst) + (FP8 ? (row * kRowBytes + ch * 16) : swz<D>(row, ch));
-    if (off >= 0) {
-      const uint8_t *src = (kv ? vbase : kbase) + off * kElemBytes + ch * 16;
-      cp_async16(dst, src);
-    } else {
-      *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-    }
-  }
-}
-
-// fp8 landing rows -> swizzled bf16 rows (exact: every E4M3 value is a bf16).
-template <int D>
-__device__ __forceinline__ void convert_fp8_stage(const uint8_t *raw, uint8_t *dst) {
-  constexpr int kChunks = kStageTokens * D / 8;  // 8 fp8 -> one 16-byte bf16 chunk
-  for (int it = threadIdx.x; it < kChunks; it += kThreads) {
-    const int row = it / (D / 8), ch = it % (D / 8);
-    const uint2 v = *reinterpret_cast<const uint2 *>(raw + row * D + ch * 8);
-    uint32_t w[2] = {v.x, v.y};
-    uint32_t outw[4];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const __nv_fp8x2_storage_t lo = (__nv_fp8x2_storage_t)(w[j] & 0xffffu);
-      const __nv_fp8x2_storage_t hi = (__nv_fp8x2_storage_t)(w[j] >> 16);
-      const float2 flo = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(lo, __NV_E4M3)));
-      const float2 fhi = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(hi, __NV_E4M3)));
-      outw[2 * j] = pack_bf16(flo.x, flo.y);
-      outw[2 * j + 1] = pack_bf16(fhi.x, fhi.y);
-    }
-    *reinterpret_cast<uint4 *>(dst + swz<D>(row, ch)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-  }
-}
-
-template <int D, int MT, bool FP8>
-__global__ void __launch_bounds__(kThreads) sparse_decode_mma_kernel(Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  using SM = MmaSmem<D, MT, FP8>;
-  SM &sm = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  const int chunk = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  Plan &pl = sm.pl;
-  if (warp == 0) make_plan(p, r, chunk, pl);
-  __syncthreads();
-  if (chunk == 0) write_empty_splits<D>(p, pl, r, g);
-  if (!pl.active) return;
-
-  fill_meta<D>(p, pl, r, g, sm.tm);
-  // Q rows m = t*G + j (head g*G + j of query token t), zero-padded to MT*16
-  {
-    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
-    for (int it = tid; it < MT * 16 * (D / 8); it += kThreads) {
-      const int m = it / (D / 8), ch = it % (D / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (m < p.M) {
-        const int t = m / p.G, h = g * p.G + m % p.G;
-        v = *reinterpret_cast<const uint4 *>(q + (((long long)r * p.T + t) * p.Hq + h) * D + ch * 8);
-      }
-      *reinterpret_cast<uint4 *>(sm.q + swz<D>(m, ch)) = v;
-    }
-  }
-  __syncthreads();
-
-  // stages of 16 micro-blocks (64 tokens)
-  const int n_stage = (pl.e_end - pl.e_begin + (kStageTokens / 4) - 1) / (kStageTokens / 4);
-
-  auto issue = [&](int st) {
-    const int buf = st & 1;
-    if (FP8)
-      load_stage<D, true>(p, sm.raw[buf][0], sm.raw[buf][1], sm.tm, st);
-    else
-      load_stage<D, false>(p, sm.kv[buf][0], sm.kv[buf][1], sm.tm, st);
-    cp_async_commit();
-  };
-
-  float o[MT][D / 8][4];
-  float mrow[MT][2], lrow[MT][2];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) o[mt][j][0] = o[mt][j][1] = o[mt][j][2] = o[mt][j][3] = 0.f;
-    mrow[mt][0] = mrow[mt][1] = -INFINITY;
-    lrow[mt][0] = lrow[mt][1] = 0.f;
-  }
-  const int gq = lane >> 2, cq = lane & 3;
-  const int p0 = pl.p0;
-
-  issue(0);
-  for (int st = 0; st < n_stage; ++st) {
-    const int buf = st & 1;
-    if (st + 1 < n_stage) {
-      issue(st + 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    if (FP8) {
-      convert_fp8_stage<D>(sm.raw[buf][0], sm.kv[buf][0]);
-      convert_fp8_stage<D>(sm.raw[buf][1], sm.kv[buf][1]);
-      __syncthreads();
-    }
-    const uint8_t *ks = sm.kv[buf][0];
-    const uint8_t *vs = sm.kv[buf][1];
-    const int tok0 = warp * 16;  // this warp's 16 tokens of the stage
-
-    // ---- S = Q K^T
-    float s[MT][2][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) s[mt][nt][0] = s[mt][nt][1] = s[mt][nt][2] = s[mt][nt][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t b0, b1, b2, b3;
-      {
-        const int row = tok0 + (lane & 7) + 8 * (lane >> 4);
-        const int ch = 2 * kk + ((lane >> 3) & 1);
-        ldsm_x4(b0, b1, b2, b3, ks + swz<D>(row, ch));
-      }
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        uint32_t a0, a1, a2, a3;
-        const int row = mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int ch = 2 * kk + (lane >> 4);
-        ldsm_x4(a0, a1, a2, a3, sm.q + swz<D>(row, ch));
-        mma_bf16(s[mt][0], a0, a1, a2, a3, b0, b1);
-        mma_bf16(s[mt][1], a0, a1, a2, a3, b2, b3);
-      }
-    }
-
-    // ---- mask, online softmax, P (hi/lo)
-    uint32_t phi[MT][4], plo[MT][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {  // row gq (hr = 0) or gq + 8 (hr = 1)
-        const int m = mt * 16 + gq + 8 * hr;
-        const int t = m / p.G;
-        const bool row_ok = m < p.M;
-        const int pt = p0 + t;
-        float x[4];
-        float mx = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int slot = st * kStageTokens + tok0 + nt * 8 + 2 * cq + e;
-            const int pos = sm.tm.pos[slot];
-            const bool ok = row_ok && pos >= 0 && pos <= pt && (sm.tm.insel[slot] || pos > p0);
-            float v = s[mt][nt][2 * hr + e] * p.scale_log2;
-            if (FP8) v *= sm.tm.ks[slot];
-            v = ok ? v : -INFINITY;
-            x[nt * 2 + e] = v;
-            mx = fmaxf(mx, v);
-          }
-        }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_old = mrow[mt][hr];
-        const float m_new = fmaxf(m_old, mx);
-        const float base = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = ex2(m_old - base);  // m_old = -inf -> 0
-        mrow[mt][hr] = m_new;
-        float psum = 0.f;
-        float pv[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float pj = ex2(x[j] - base);
-          psum += pj;
-          const int slot = st * kStageTokens + tok0 + (j >> 1) * 8 + 2 * cq + (j & 1);
-          pv[j] = FP8 ? pj * sm.tm.vs[slot] : pj;
-        }
-        lrow[mt][hr] = lrow[mt][hr] * alpha + psum;
-#pragma unroll
-        for (int dt = 0; dt < D / 8; ++dt) {
-          o[mt][dt][2 * hr] *= alpha;
-          o[mt][dt][2 * hr + 1] *= alpha;
-        }
-        // A fragment regs: a0 (row gq, k 2cq..) = nt0 e0,e1 ; a1 (row gq+8) ; a2 (row gq, k+8) = nt1 ; a3
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const float v0 = pv[nt * 2], v1 = pv[nt * 2 + 1];
-          const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-          const float2 hf = __bfloat1622float2(h);
-          const uint32_t hw = *reinterpret_cast<const uint32_t *>(&h);
-          const uint32_t lw = pack_bf16(v0 - hf.x, v1 - hf.y);
-          phi[mt][nt * 2 + hr] = hw;
-          plo[mt][nt * 2 + hr] = lw;
-        }
-      }
-    }
-
-    // ---- O += P V
-#pragma unroll
-    for (int dp = 0; dp < D / 16; ++dp) {
-      uint32_t v0, v1, v2, v3;
-      {
-        const int row = tok0 + (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int ch = 2 * dp + (lane >> 4);
-        ldsm_x4_t(v0, v1, v2, v3, vs + swz<D>(row, ch));
-      }
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        // A regs order: a0 = (row g, k lo) = phi[0], a1 = (row g+8, k lo) = phi[1],
-        //               a2 = (row g, k hi) = phi[2], a3 = (row g+8, k hi) = phi[3]
-        mma_bf16(o[mt][2 * dp], phi[mt][0], phi[mt][1], phi[mt][2], phi[mt][3], v0, v1);
-        mma_bf16(o[mt][2 * dp], plo[mt][0], plo[mt][1], plo[mt][2], plo[mt][3], v0, v1);
-        mma_bf16(o[mt][2 * dp + 1], phi[mt][0], phi[mt][1], phi[mt][2], phi[mt][3], v2, v3);
-        mma_bf16(o[mt][2 * dp + 1], plo[mt][0], plo[mt][1], plo[mt][2], plo[mt][3], v2, v3);
-      }
-    }
-    __syncthreads();  // buffer `buf` may be refilled by the next issue
-  }
-
-  // ---- merge the four warps' states
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      float l = lrow[mt][hr];
-      l += __shfl_xor_sync(0xffffffffu, l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      lrow[mt][hr] = l;
-      if (cq == 0) {
-        sm.wm[warp][mt * 16 + gq + 8 * hr] = mrow[mt][hr];
-        sm.wl[warp][mt * 16 + gq + 8 * hr] = l;
-      }
-    }
-  __syncthreads();
-  // per-warp rescaled O into shared memory (reuses the K/V buffers)
-  float *ow = reinterpret_cast<float *>(&sm.kv[0][0][0]);  // [kWarps][MT*16][D]
-  static_assert(sizeof(sm.kv) >= sizeof(float) * kWarps * MT * 16 * D, "O staging fits");
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      const int m = mt * 16 + gq + 8 * hr;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, sm.wm[w][m]);
-      const float f = (mx == -INFINITY) ? 0.f : exp2f(mrow[mt][hr] - mx);
-#pragma unroll
-      for (int dt = 0; dt < D / 8; ++dt) {
-        float *dst = ow + ((warp * MT * 16) + m) * D + dt * 8 + 2 * cq;
-        dst[0] = o[mt][dt][2 * hr] * f;
-        dst[1] = o[mt][dt][2 * hr + 1] * f;
-      }
-    }
-  __syncthreads();
-  // final o (normalised) into warp 0's block, lse into sm.lse; element (m, d)
-  // is read and rewritten by the same thread only
-  for (int i = tid; i < p.M * D; i += kThreads) {
-    const int m = i / D, d = i % D;
-    float mx = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, sm.wm[w][m]);
-    float den = 0.f, num = 0.f;
-    if (mx != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        den += sm.wl[w][m] * exp2f(sm.wm[w][m] - mx);
-        num += ow[(w * MT * 16 + m) * D + d];
-      }
-    }
-    ow[m * D + d] = den > 0.f ? num / den : 0.f;
-    if (d == 0) sm.lse[m] = den > 0.f ? (mx + __log2f(den)) * kLn2 : -INFINITY;
-  }
-  __syncthreads();
-  finish_chunk<D>(p, pl, r, g, ow, sm.lse, &sm.flag, ow + p.M * D);
 }
 
 // ------------------------------------------------------- fp32 K/V path --

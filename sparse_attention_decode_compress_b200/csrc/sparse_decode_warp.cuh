@@ -1,0 +1,457 @@
+// qsa_sparse_decode, BF16 / FP8 caches: persistent warp-level split-KV
+// flash-decoding on mma.sync bf16 tiles.
+//
+// Chunks of the extended selection inside each split (sparse_decode.cuh),
+// online softmax in fp32, P fed to the PV product as a bf16 hi + lo pair
+// (two MMAs, ~16 significant bits), LSE merge of a split's chunks by the
+// last chunk to finish.  FP8 E4M3 rows are converted to bf16 in shared
+// memory (exact); the per-(page, head) K scale multiplies the logits and the
+// V scale multiplies P.  Organised for memory-level parallelism on
+// B200: one CTA of NW warps per SM, each warp an independent worker that
+// takes (request, kv head, chunk) items from an atomic counter and streams
+// its chunk through its own ring of NS 16-token K/V stages with cp.async
+// (NS - 1 stages in flight while one is computed).  No CTA
+// barriers: warps never wait for each other, results go straight from the
+// MMA accumulators to global memory.
+#pragma once
+#include "sparse_decode.cuh"
+
+namespace qsa {
+namespace dec {
+
+constexpr int kTokW = 16;         // tokens per stage
+constexpr int kCounterInts = 64;  // workspace header: [0] next item, [1] finished warps
+
+// Shared-memory layout of one worker warp: a ring of NS 16-token K/V stages,
+// an fp8 -> bf16 conversion stage and the chunk's token metadata.
+template <int D, bool FP8, int NS>
+struct WarpState {
+  static constexpr int kRowBytes = D * (FP8 ? 1 : 2);
+  alignas(128) uint8_t ring[NS][2][kTokW * kRowBytes];
+  alignas(128) uint8_t cvt[FP8 ? 2 : 1][FP8 ? kTokW * D * 2 : 16];
+  int off[kChunkTokens];             // (token, head) row index in the cache, -1 = nothing to load
+  unsigned char vmask[kChunkTokens]; // bit t: the token is visible to query token t
+  float ks[FP8 ? kChunkTokens : 1];
+  float vs[FP8 ? kChunkTokens : 1];
+  Plan pl;
+};
+
+template <int D, bool FP8, int NW, int NS>
+struct WarpSmem {
+  WarpState<D, FP8, NS> w[NW];
+};
+
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Warp-level: empty splits of (r, g) get o = 0, lse = -inf.
+template <int D>
+__device__ void write_empty_splits_warp(const Params &p, const Plan &pl, int r, int g, int lane) {
+  for (int s = 0; s < p.S; ++s) {
+    if (pl.ch_count[s] != 0) continue;
+    for (int i = lane; i < p.M * D; i += 32) {
+      const int m = i / D, d = i % D;
+      p.o_part[out_row(p, s, r, g, m) * D + d] = 0.f;
+      if (d == 0) p.lse_part[out_row(p, s, r, g, m)] = -INFINITY;
+    }
+  }
+}
+
+// Token metadata of the chunk: cache row, visibility bits and fp8 scales.
+// Token i is visible to query token t (position p_t = p0 + t) when i <= p_t
+// and (its block is selected or i > p0).
+template <typename WS, bool FP8>
+__device__ void fill_meta_warp(const Params &p, const Plan &pl, int r, int g, WS &W, int lane) {
+  const int32_t *sel_r = p.sel + (long long)r * p.topk;
+  const int P = p.c.page_size, Hkv = p.c.num_kv_heads;
+  int bl[kChunkTokens / 32];
+#pragma unroll
+  for (int i = 0; i < kChunkTokens / 32; ++i) {
+    const int k = lane + 32 * i;
+    const int e = pl.e_begin + k / 4;
+    bl[i] = (e < pl.e_end) ? ext_block(sel_r, pl, e) : -1;
+  }
+#pragma unroll
+  for (int i = 0; i < kChunkTokens / 32; ++i) {
+    const int k = lane + 32 * i;
+    const int b = bl[i];
+    int off = -1;
+    unsigned vm = 0;
+    float ks = 1.f, vs = 1.f;
+    if (b >= 0) {
+      const long long t = 4LL * b + (k & 3);
+      if (t < pl.L) {
+        const int page = physical_page(p.c, r, t / P);
+        if (page >= 0) {
+          off = (int)(((long long)page * P + (t % P)) * Hkv + g);
+          const bool ins = (pl.e_begin + k / 4) < pl.nvalid;
+          for (int q = 0; q < p.T; ++q)
+            if (t <= (long long)pl.p0 + q && (ins || t > pl.p0)) vm |= 1u << q;
+          if (FP8) {
+            ks = p.c.k_scale[(long long)page * Hkv + g];
+            vs = p.c.v_scale[(long long)page * Hkv + g];
+          }
+        }
+      } else if ((k & 3) == 0 && 4LL * b >= pl.L) {
+        record_error(kErrBadInput);  // selected block beyond the context
+      }
+    }
+    W.off[k] = off;
+    W.vmask[k] = (unsigned char)vm;
+    if (FP8) {
+      W.ks[k] = ks;
+      W.vs[k] = vs;
+    }
+  }
+}
+
+// cp.async of stage st of the chunk into ring slot `slot` (rows swizzled for
+// bf16; fp8 rows land raw and are converted before use).
+template <int D, bool FP8, typename WS>
+__device__ __forceinline__ void issue_stage_warp(const Params &p, WS &W, int slot, int st,
+                                                 int lane) {
+  constexpr int kRowBytes = WS::kRowBytes;
+  constexpr int kCh = kRowBytes / 16;  // 16-byte chunks per row
+  constexpr int kItems = 2 * kTokW * kCh;
+  const uint8_t *kbase = static_cast<const uint8_t *>(p.c.k_cache);
+  const uint8_t *vbase = static_cast<const uint8_t *>(p.c.v_cache);
+#pragma unroll
+  for (int i = 0; i < kItems / 32; ++i) {
+    const int it = lane + 32 * i;
+    const int kv = it / (kTokW * kCh);
+    const int rem = it % (kTokW * kCh);
+    const int row = rem / kCh, ch = rem % kCh;
+    const int off = W.off[st * kTokW + row];
+    uint8_t *dst = W.ring[slot][kv] + (FP8 ? (row * kRowBytes + ch * 16) : swz<D>(row, ch));
+    if (off >= 0) {
+      cp_async16(dst, (kv ? vbase : kbase) + (long long)off * kRowBytes + ch * 16);
+    } else {
+      *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void convert_fp8_rows_warp(const uint8_t *raw, uint8_t *dst, int lane) {
+  constexpr int kChunks = kTokW * D / 8;
+#pragma unroll
+  for (int i = 0; i < kChunks / 32; ++i) {
+    const int it = lane + 32 * i;
+    const int row = it / (D / 8), ch = it % (D / 8);
+    const uint2 v = *reinterpret_cast<const uint2 *>(raw + row * D + ch * 8);
+    const uint32_t w[2] = {v.x, v.y};
+    uint32_t outw[4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const __nv_fp8x2_storage_t lo = (__nv_fp8x2_storage_t)(w[j] & 0xffffu);
+      const __nv_fp8x2_storage_t hi = (__nv_fp8x2_storage_t)(w[j] >> 16);
+      const float2 flo = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(lo, __NV_E4M3)));
+      const float2 fhi = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(hi, __NV_E4M3)));
+      outw[2 * j] = pack_bf16(flo.x, flo.y);
+      outw[2 * j + 1] = pack_bf16(fhi.x, fhi.y);
+    }
+    *reinterpret_cast<uint4 *>(dst + swz<D>(row, ch)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+  }
+}
+
+// Tensor-core decode, tokens on M: per 16-token stage
+//   S^T[16 tokens x 8*NT rows] = K[16 x D] . Q^T          (mma m16n8k16, A = K
+//                                                          from smem, B = Q in
+//                                                          registers)
+//   P^T = exp2(S^T * scale - m) per query row (a column here); transposed to
+//         the B layout of the next product with movmatrix, as bf16 hi + lo
+//   O^T[D x 8*NT] += V^T[D x 16 tokens] . P^T              (A = V rows loaded
+//                                                          with ldmatrix.trans)
+// Query rows m = t*G + j (head g*G + j of query token t) sit on the N side in
+// tiles of 8, so G*T = 8 uses every MMA lane.
+template <int D, int NT, bool FP8, int NW, int NS>
+__global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  using SM = WarpSmem<D, FP8, NW, NS>;
+  using WS = WarpState<D, FP8, NS>;
+  SM &sm = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  WS &W = sm.w[warp];
+  Plan &pl = W.pl;
+  const int Hkv = p.c.num_kv_heads;
+  const int total_items = p.B * Hkv * p.nch;
+  const int gq = lane >> 2, cq = lane & 3;
+  constexpr int MD = D / 16;  // m-tiles of O^T (16 dims each)
+
+  while (true) {
+    int it = 0;
+    if (lane == 0) it = atomicAdd(&p.counters[0], 1);
+    it = __shfl_sync(0xffffffffu, it, 0);
+    if (it >= total_items) break;
+    const int c = it % p.nch;
+    const int g = (it / p.nch) % Hkv;
+    const int r = it / (p.nch * Hkv);
+    make_plan(p, r, c, pl);
+    __syncwarp();
+    if (c == 0) write_empty_splits_warp<D>(p, pl, r, g, lane);
+    if (!pl.active) continue;
+    fill_meta_warp<WS, FP8>(p, pl, r, g, W, lane);
+
+    // Q as B fragments: n-tile j, k-step kk: b0 = Q[row 8j+gq][16kk+2cq, +1],
+    // b1 = Q[row 8j+gq][16kk+2cq+8, +9]; rows >= M are zero
+    uint32_t qb[NT][MD][2];
+    {
+      const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const int m = 8 * j + gq;
+        const bool ok = m < p.M;
+        const __nv_bfloat16 *qrow =
+            qg + (((long long)r * p.T + (ok ? m / p.G : 0)) * p.Hq + g * p.G + (ok ? m % p.G : 0)) * D;
+#pragma unroll
+        for (int kk = 0; kk < MD; ++kk) {
+          qb[j][kk][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq) : 0u;
+          qb[j][kk][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq + 8) : 0u;
+        }
+      }
+    }
+    // query token of each of this lane's columns (rows 8j + 2cq + e); -1 = padding
+    int tcol[NT][2];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int m = 8 * j + 2 * cq + e;
+        tcol[j][e] = m < p.M ? m / p.G : -1;
+      }
+    __syncwarp();
+
+    const int nst = (pl.e_end - pl.e_begin + 3) / 4;  // 4 micro-blocks per stage
+    float o[MD][NT][4];
+    float mcol[NT][2], lcol[NT][2];
+#pragma unroll
+    for (int i = 0; i < MD; ++i)
+#pragma unroll
+      for (int j = 0; j < NT; ++j) o[i][j][0] = o[i][j][1] = o[i][j][2] = o[i][j][3] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      mcol[j][0] = mcol[j][1] = -INFINITY;
+      lcol[j][0] = lcol[j][1] = 0.f;
+    }
+#pragma unroll
+    for (int s0 = 0; s0 < NS - 1; ++s0) {
+      if (s0 < nst) issue_stage_warp<D, FP8>(p, W, s0, s0, lane);
+      cp_async_commit();
+    }
+    for (int st = 0; st < nst; ++st) {
+      {
+        const int sn = st + NS - 1;
+        if (sn < nst) issue_stage_warp<D, FP8>(p, W, sn % NS, sn, lane);
+        cp_async_commit();
+      }
+      cp_async_wait<NS - 1>();
+      __syncwarp();
+      const int slot = st % NS;
+      const uint8_t *ks_t;
+      const uint8_t *vs_t;
+      if constexpr (FP8) {
+        convert_fp8_rows_warp<D>(W.ring[slot][0], W.cvt[0], lane);
+        convert_fp8_rows_warp<D>(W.ring[slot][1], W.cvt[1], lane);
+        __syncwarp();
+        ks_t = W.cvt[0];
+        vs_t = W.cvt[1];
+      } else {
+        ks_t = W.ring[slot][0];
+        vs_t = W.ring[slot][1];
+      }
+      const int tb = st * kTokW;  // chunk index of the stage's first token
+
+      // ---- S^T = K Q^T
+      float sacc[NT][4];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < MD; ++kk) {
+        uint32_t a0, a1, a2, a3;
+        {
+          const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+          const int ch = 2 * kk + (lane >> 4);
+          ldsm_x4(a0, a1, a2, a3, ks_t + swz<D>(row, ch));
+        }
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma_bf16(sacc[j], a0, a1, a2, a3, qb[j][kk][0], qb[j][kk][1]);
+      }
+
+      // ---- mask, online softmax per column, P^T as bf16 hi + lo B fragments
+      const unsigned vm0 = W.vmask[tb + gq], vm1 = W.vmask[tb + gq + 8];
+      float ksc0 = 1.f, ksc1 = 1.f, vsc0 = 1.f, vsc1 = 1.f;
+      if constexpr (FP8) {
+        ksc0 = W.ks[tb + gq];
+        ksc1 = W.ks[tb + gq + 8];
+        vsc0 = W.vs[tb + gq];
+        vsc1 = W.vs[tb + gq + 8];
+      }
+      uint32_t bhi[NT][2], blo[NT][2];
+      bool rescale = false;
+      float alpha[NT][2];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = tcol[j][e];
+          const bool ok0 = t >= 0 && ((vm0 >> t) & 1u);
+          const bool ok1 = t >= 0 && ((vm1 >> t) & 1u);
+          x[e] = ok0 ? sacc[j][e] * p.scale_log2 * ksc0 : -INFINITY;      // token gq
+          x[2 + e] = ok1 ? sacc[j][2 + e] * p.scale_log2 * ksc1 : -INFINITY;  // token gq+8
+        }
+        float pj[4];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float mx = fmaxf(x[e], x[2 + e]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float m_old = mcol[j][e];
+          const float m_new = fmaxf(m_old, mx);
+          const float base = (m_new == -INFINITY) ? 0.f : m_new;
+          const float a = (m_new == -INFINITY) ? 1.f : ex2(m_old - base);  // empty column: keep
+          alpha[j][e] = a;
+          rescale |= (a != 1.f);
+          mcol[j][e] = m_new;
+          pj[e] = ex2(x[e] - base);
+          pj[2 + e] = ex2(x[2 + e] - base);
+          lcol[j][e] = lcol[j][e] * a + pj[e] + pj[2 + e];  // this lane's two tokens
+        }
+        const float v0 = pj[0] * vsc0, v1 = pj[1] * vsc0, v2 = pj[2] * vsc1, v3 = pj[3] * vsc1;
+        const __nv_bfloat162 h01 = __floats2bfloat162_rn(v0, v1);
+        const __nv_bfloat162 h23 = __floats2bfloat162_rn(v2, v3);
+        const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+        // tile of tokens 0-7 (lane holds token gq, cols 2cq..) -> b0; tokens 8-15 -> b1
+        bhi[j][0] = movmatrix_t(*reinterpret_cast<const uint32_t *>(&h01));
+        bhi[j][1] = movmatrix_t(*reinterpret_cast<const uint32_t *>(&h23));
+        blo[j][0] = movmatrix_t(pack_bf16(v0 - f01.x, v1 - f01.y));
+        blo[j][1] = movmatrix_t(pack_bf16(v2 - f23.x, v3 - f23.y));
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int i = 0; i < MD; ++i)
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            o[i][j][0] *= alpha[j][0];
+            o[i][j][1] *= alpha[j][1];
+            o[i][j][2] *= alpha[j][0];
+            o[i][j][3] *= alpha[j][1];
+          }
+      }
+
+      // ---- O^T += V^T P^T
+#pragma unroll
+      for (int i = 0; i < MD; ++i) {
+        uint32_t a0, a1, a2, a3;
+        {
+          const int row = (lane & 7) + 8 * (lane >> 4);
+          const int ch = 2 * i + ((lane >> 3) & 1);
+          ldsm_x4_t(a0, a1, a2, a3, vs_t + swz<D>(row, ch));
+        }
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          mma_bf16(o[i][j], a0, a1, a2, a3, bhi[j][0], bhi[j][1]);
+          mma_bf16(o[i][j], a0, a1, a2, a3, blo[j][0], blo[j][1]);
+        }
+      }
+      __syncwarp();  // the slot may be refilled by the next issue
+    }
+    cp_async_wait<0>();
+
+    // ---- chunk result: column sums over the 8 token lanes, then o and lse
+    const int s_idx = pl.split;
+    const bool direct = pl.nchunks_split == 1;
+    const long long wslot = ((long long)r * Hkv + g) * p.nch + c;
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float l = lcol[j][e];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        const int m = 8 * j + 2 * cq + e;
+        if (m >= p.M) continue;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        float *orow = direct ? p.o_part + out_row(p, s_idx, r, g, m) * D : p.ws_o + (wslot * p.M + m) * D;
+#pragma unroll
+        for (int i = 0; i < MD; ++i) {
+          orow[16 * i + gq] = o[i][j][e] * inv;
+          orow[16 * i + gq + 8] = o[i][j][2 + e] * inv;
+        }
+        if (gq == 0) {
+          const float lse = l > 0.f ? (mcol[j][e] + __log2f(l)) * kLn2 : -INFINITY;
+          if (direct) p.lse_part[out_row(p, s_idx, r, g, m)] = lse;
+          else p.ws_lse[wslot * p.M + m] = lse;
+        }
+      }
+    if (direct) continue;
+
+    // ---- several chunks in this split: the last to finish merges them
+    __threadfence();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      int32_t *ticket = p.tickets + ((long long)r * Hkv + g) * p.S + s_idx;
+      const int t = atomicAdd(ticket, 1);
+      last = (t == pl.nchunks_split - 1);
+      if (last) *ticket = 0;
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) continue;
+    __threadfence();
+    const long long slot0 = ((long long)r * Hkv + g) * p.nch + pl.first_chunk_of_split;
+    const int nc = pl.nchunks_split;
+    float *lse_c = reinterpret_cast<float *>(&W.ring[0][0][0]);  // [nc][M], ring is idle now
+    for (int i = lane; i < nc * p.M; i += 32) lse_c[i] = __ldcg(p.ws_lse + slot0 * p.M + i);
+    __syncwarp();
+    for (int e4 = lane; e4 < p.M * D / 4; e4 += 32) {
+      const int m = (e4 * 4) / D, d = (e4 * 4) % D;
+      float mx = -INFINITY;
+      for (int cc = 0; cc < nc; ++cc) mx = fmaxf(mx, lse_c[cc * p.M + m]);
+      float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+      float den = 0.f;
+      if (mx != -INFINITY) {
+        for (int cc = 0; cc < nc; cc += 4) {
+          float4 ov[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            ov[u] = (cc + u < nc) ? __ldcg(reinterpret_cast<const float4 *>(
+                                        p.ws_o + ((slot0 + cc + u) * p.M + m) * D + d))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (cc + u >= nc) break;
+            const float l = lse_c[(cc + u) * p.M + m];
+            const float w = (l == -INFINITY) ? 0.f : __expf(l - mx);
+            den += w;
+            num.x += w * ov[u].x;
+            num.y += w * ov[u].y;
+            num.z += w * ov[u].z;
+            num.w += w * ov[u].w;
+          }
+        }
+      }
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      *reinterpret_cast<float4 *>(p.o_part + out_row(p, s_idx, r, g, m) * D + d) =
+          make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+      if (d == 0) p.lse_part[out_row(p, s_idx, r, g, m)] = den > 0.f ? mx + __logf(den) : -INFINITY;
+    }
+    __syncwarp();
+  }
+  // every warp reports once; the last one resets the work counters
+  if (lane == 0) {
+    const int total_warps = gridDim.x * NW;
+    if (atomicAdd(&p.counters[1], 1) == total_warps - 1) {
+      atomicExch(&p.counters[0], 0);
+      atomicExch(&p.counters[1], 0);
+    }
+  }
+}
+
+}  // namespace dec
+}  // namespace qsa
