@@ -71,7 +71,7 @@ __device__ __forceinline__ uint32_t score_key(int s) {
 // by the scan kernel, L2-resident) are read with 16-byte loads issued in
 // batches of kSelBatch per thread, so many loads are in flight at once.
 
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = 1024;
 constexpr int kSelBatch = 8;  // int4 loads in flight per thread
 
 struct SelSmem {

@@ -66,6 +66,8 @@ struct Plan {
   int active;  // this CTA owns a chunk
   int e_bound[kMaxSplits + 1];
   int ch_count[kMaxSplits];
+  long long tb[kMaxSplits + 1];  // token boundary of each split
+  int cnt[kMaxSplits];           // selected blocks per split
 };
 
 // Entry k of the extended selection of request r.
@@ -73,9 +75,10 @@ __device__ __forceinline__ int ext_block(const int32_t *sel_r, const Plan &pl, i
   return k < pl.nvalid ? sel_r[k] : pl.extra[k - pl.nvalid];
 }
 
-// Warp 0 reads the selection row once, coalesced (32 entries per load), and
-// counts, per split boundary, the selected blocks that start before it; the
-// list is ascending, so those counts are the boundaries in the extended list.
+// One warp reads the selection row once, coalesced, and counts the selected
+// blocks of every split (split of a block: binary search of its first token
+// in the split boundaries); the list is ascending, so the running counts are
+// the split boundaries in the extended list.
 __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl) {
   const int lane = threadIdx.x & 31;
   const int32_t *sel_r = p.sel + (long long)r * p.topk;
@@ -86,36 +89,32 @@ __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl) {
   }
   const int p0 = L - p.T;
   const long long NP = ((long long)L + p.c.page_size - 1) / p.c.page_size;
-  // token boundary of split s (lane s holds boundary s, s = 1 .. S-1)
-  long long tb = 0;
-  if (lane >= 1 && lane < p.S) tb = min(((long long)lane * NP / p.S) * p.c.page_size, (long long)L);
+  if (lane <= p.S) pl.tb[lane] = min(((long long)lane * NP / p.S) * p.c.page_size, (long long)L);
+  if (lane < p.S) pl.cnt[lane] = 0;
+  __syncwarp();
   int nvalid = 0, last = -1;
-  int below[kMaxSplits];  // below[s]: selected blocks starting before boundary s
-#pragma unroll
-  for (int s = 0; s < kMaxSplits; ++s) below[s] = 0;
   const int n_entries = (L > 0) ? p.topk : 0;
-  for (int base = 0; base < n_entries; base += 32 * 8) {
-    int v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int k = base + j * 32 + lane;
-      v[j] = (k < n_entries) ? sel_r[k] : -1;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const bool valid = v[j] >= 0;
-      nvalid += __popc(__ballot_sync(0xffffffffu, valid));
-      last = max(last, v[j]);
-#pragma unroll
-      for (int s = 1; s < kMaxSplits; ++s) {
-        if (s >= p.S) break;
-        const long long tbs = __shfl_sync(0xffffffffu, tb, s);
-        below[s] += __popc(__ballot_sync(0xffffffffu, valid && 4LL * v[j] < tbs));
+  for (int k = lane; k < n_entries; k += 32) {
+    const int v = sel_r[k];
+    const bool valid = v >= 0;
+    nvalid += __popc(__ballot_sync(__activemask(), valid));
+    if (valid) {
+      last = max(last, v);
+      const long long t = 4LL * v;
+      int lo = 0, hi = p.S;  // split s with tb[s] <= t < tb[s+1]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pl.tb[mid] <= t) lo = mid; else hi = mid;
       }
+      atomicAdd(&pl.cnt[lo], 1);
     }
   }
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+  for (int o = 16; o >= 1; o >>= 1) {
+    last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+    nvalid = max(nvalid, __shfl_xor_sync(0xffffffffu, nvalid, o));
+  }
+  __syncwarp();
   if (lane == 0) {
     pl.L = L;
     pl.p0 = p0;
@@ -129,19 +128,15 @@ __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl) {
     }
     pl.n_extra = ne;
     pl.nE = nvalid + ne;
-    pl.e_bound[0] = 0;
-    pl.e_bound[p.S] = pl.nE;
-#pragma unroll
-    for (int s = 1; s < kMaxSplits; ++s) {
-      if (s < p.S) {
-        const long long tbs = min(((long long)s * NP / p.S) * p.c.page_size, (long long)L);
-        int eb = below[s];
-        for (int x = 0; x < ne; ++x) eb += (4LL * pl.extra[x] < tbs);
-        pl.e_bound[s] = eb;
-      }
-    }
     int cum = 0;
     pl.active = 0;
+    pl.e_bound[0] = 0;
+    for (int s = 0; s < p.S; ++s) {
+      int n = pl.cnt[s];
+      for (int x = 0; x < ne; ++x)
+        n += (4LL * pl.extra[x] >= pl.tb[s] && 4LL * pl.extra[x] < pl.tb[s + 1]);
+      pl.e_bound[s + 1] = pl.e_bound[s] + n;
+    }
     for (int s = 0; s < p.S; ++s) {
       const int n = pl.e_bound[s + 1] - pl.e_bound[s];
       const int ch = (n + kChunkBlocks - 1) / kChunkBlocks;

@@ -126,11 +126,8 @@ __device__ __forceinline__ void issue_stage_warp(const Params &p, WS &W, int slo
     const int row = rem / kCh, ch = rem % kCh;
     const int off = W.off[st * kTokW + row];
     uint8_t *dst = W.ring[slot][kv] + (FP8 ? (row * kRowBytes + ch * 16) : swz<D>(row, ch));
-    if (off >= 0) {
-      cp_async16(dst, (kv ? vbase : kbase) + (long long)off * kRowBytes + ch * 16);
-    } else {
-      *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-    }
+    const uint8_t *src = (kv ? vbase : kbase) + (long long)max(off, 0) * kRowBytes + ch * 16;
+    cp_async16_zfill(dst, src, off >= 0);
   }
 }
 
@@ -264,10 +261,12 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p
       }
       const int tb = st * kTokW;  // chunk index of the stage's first token
 
-      // ---- S^T = K Q^T
-      float sacc[NT][4];
+      // ---- S^T = K Q^T (even and odd k-steps in two accumulators: shorter chains)
+      float sacc[NT][4], sac2[NT][4];
 #pragma unroll
-      for (int j = 0; j < NT; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[j][e] = sac2[j][e] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < MD; ++kk) {
         uint32_t a0, a1, a2, a3;
@@ -277,8 +276,15 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p
           ldsm_x4(a0, a1, a2, a3, ks_t + swz<D>(row, ch));
         }
 #pragma unroll
-        for (int j = 0; j < NT; ++j) mma_bf16(sacc[j], a0, a1, a2, a3, qb[j][kk][0], qb[j][kk][1]);
+        for (int j = 0; j < NT; ++j) {
+          if (kk & 1) mma_bf16(sac2[j], a0, a1, a2, a3, qb[j][kk][0], qb[j][kk][1]);
+          else mma_bf16(sacc[j], a0, a1, a2, a3, qb[j][kk][0], qb[j][kk][1]);
+        }
       }
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[j][e] += sac2[j][e];
 
       // ---- mask, online softmax per column, P^T as bf16 hi + lo B fragments
       const unsigned vm0 = W.vmask[tb + gq], vm1 = W.vmask[tb + gq + 8];
