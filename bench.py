@@ -42,7 +42,7 @@ def parse_args(argv=None):
                     help="override the workload's batch (profiling runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-queries", type=int, default=8,
+    ap.add_argument("--cpu-queries", type=int, default=300,
                     help="oracle queries timed for the CPU baseline")
     return ap.parse_args(argv)
 

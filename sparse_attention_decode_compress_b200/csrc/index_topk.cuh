@@ -81,25 +81,6 @@ struct SelSmem {
   int bin, above, nkeep, ncand, fb_key, fb_above, fb_idx;
 };
 
-__device__ __forceinline__ void bitonic_sort_u64(unsigned long long *a, int n_pow2, int tid) {
-  for (int k = 2; k <= n_pow2; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < n_pow2; i += kSelThreads) {
-        const int l = i ^ j;
-        if (l > i) {
-          const unsigned long long x = a[i], y = a[l];
-          const bool up = (i & k) == 0;
-          if ((x > y) == up) {
-            a[i] = y;
-            a[l] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-}
-
 __device__ __forceinline__ void bitonic_sort_i32(int *a, int n_pow2, int tid) {
   for (int k = 2; k <= n_pow2; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
@@ -277,6 +258,25 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
   __syncthreads();
 }
 
+// Writes the K distinct kept indices in ascending order: by rank counting
+// for small K, by a bitonic sort otherwise.
+__device__ void write_ascending(int *keep, int K, int32_t *out, SelSmem &sm, int tid) {
+  if (K <= 1024) {
+    for (int i = tid; i < K; i += kSelThreads) {
+      const int x = keep[i];
+      int rank = 0;
+      for (int j = 0; j < K; ++j) rank += (keep[j] < x);
+      out[rank] = x;
+    }
+    return;
+  }
+  const int kp2 = next_pow2(K);
+  for (int i = K + tid; i < kp2; i += kSelThreads) keep[i] = 0x7fffffff;
+  __syncthreads();
+  bitonic_sort_i32(keep, kp2, tid);
+  for (int i = tid; i < K; i += kSelThreads) out[i] = keep[i];
+}
+
 // Selection kernel: grid = B, one request per CTA.
 __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -321,22 +321,21 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
   const int above = sm.above;
   const int ncand = sm.ncand;
   if (ncand <= kCandCap) {
-    const int np2 = next_pow2(ncand);
-    for (int i = ncand + tid; i < np2; i += kSelThreads) sm.cand[i] = ~0ull;
-    __syncthreads();
-    bitonic_sort_u64(sm.cand, np2, tid);
-    for (int j = tid; j < K - above; j += kSelThreads)
-      keep[above + j] = (int)(uint32_t)(sm.cand[j] & 0xffffffffu);
+    // candidates of the threshold bin: the (K - above) first by (score desc,
+    // index asc); keys are distinct, so a candidate's rank is the number of
+    // smaller keys
+    const int need = K - above;
+    for (int i = tid; i < ncand; i += kSelThreads) {
+      const unsigned long long x = sm.cand[i];
+      int rank = 0;
+      for (int j = 0; j < ncand; ++j) rank += (sm.cand[j] < x);
+      if (rank < need) keep[above + rank] = (int)(uint32_t)(x & 0xffffffffu);
+    }
     __syncthreads();
   } else {
     select_fallback(sc, n, K, sm, tid);
   }
-  // kept indices in ascending order
-  const int kp2 = next_pow2(K);
-  for (int i = K + tid; i < kp2; i += kSelThreads) keep[i] = 0x7fffffff;
-  __syncthreads();
-  bitonic_sort_i32(keep, kp2, tid);
-  for (int i = tid; i < K; i += kSelThreads) out[i] = keep[i];
+  write_ascending(keep, K, out, sm, tid);
 }
 
 // ------------------------------------------------------------- the scan --
@@ -403,8 +402,49 @@ struct ItemWalker {
   }
 };
 
+#ifndef QSA_SCAN_MIN_CTAS
+#define QSA_SCAN_MIN_CTAS 6
+#endif
+#ifndef QSA_SCAN_LOAD
+#define QSA_SCAN_LOAD 2
+#endif
+#ifndef QSA_SCORE_STORE
+#define QSA_SCORE_STORE 1
+#endif
+// 16-byte load of compressed keys, read once per call.
+__device__ __forceinline__ uint4 scan_load(const uint4 *p, uint64_t policy) {
+  uint4 v;
+#if QSA_SCAN_LOAD == 0
+  v = __ldcs(p);
+#elif QSA_SCAN_LOAD == 1
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+#else
+  // not cached in L1, L2 evict-first (the stream does not push the scores out
+  // of L2), 256-byte L2 prefetch
+  asm volatile(
+      "ld.global.nc.L1::no_allocate.L2::cache_hint.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p), "l"(policy));
+#endif
+  return v;
+}
+// Score store; L2 evict-last keeps it for the selection kernel.
+__device__ __forceinline__ void score_store(int32_t *p, int v, uint64_t policy) {
+#if QSA_SCORE_STORE == 0
+  *p = v;
+#else
+  asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(policy) : "memory");
+#endif
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 template <int DI>
-__global__ void __launch_bounds__(kScanThreads) index_scan_kernel(Params p) {
+__global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_kernel(Params p) {
   constexpr int kLPR = DI / 8;                    // lanes per row (16 B each)
   constexpr int kRPI = 32 / kLPR;                 // rows per load instruction
   constexpr int kRowsPerItem = kItemLoads * kRPI; // 4096 / DI
@@ -417,6 +457,8 @@ __global__ void __launch_bounds__(kScanThreads) index_scan_kernel(Params p) {
   const int sub = lane % kLPR;                    // this lane's 8 dims: 8*sub .. 8*sub+7
   const int row_in = lane / kLPR;
 
+  const uint64_t pol_stream = l2_policy_evict_first();
+  const uint64_t pol_keep = l2_policy_evict_last();
   ItemWalker wk;
   wk.start(p, kRowsPerItem, warp_id == 0 && lane == 0);
   int cur_r = -1;
@@ -473,7 +515,7 @@ __global__ void __launch_bounds__(kScanThreads) index_scan_kernel(Params p) {
         if (pg >= 0) {
           const uint4 *src = reinterpret_cast<const uint4 *>(
               p.c.kc + ((long long)pg * bpp + off) * DI + sub * 8);
-          v[i] = __ldcs(src);
+          v[i] = scan_load(src, pol_stream);
         } else if (lane == 0 || sub == 0) {
           record_error(kErrBounds);
         }
@@ -507,7 +549,7 @@ __global__ void __launch_bounds__(kScanThreads) index_scan_kernel(Params p) {
     for (int k = 0; k < kVals; ++k) {
       const int i = ((lane % kLPR) << (4 - kR)) | k;
       const int row = row0 + i * kRPI + row_in;
-      if (row < n) sc[row] = acc[k];
+      if (row < n) score_store(sc + row, acc[k], pol_keep);
     }
     if (!more) break;
   }

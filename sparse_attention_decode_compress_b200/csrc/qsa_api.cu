@@ -134,10 +134,16 @@ int decode_chunk_slots(int topk, int S) {
 // Worker warps per SM and ring depth of the tensor-core decode kernel: as
 // many warps as registers allow (query-row tiles NT set the accumulator
 // size), then as deep a ring as shared memory allows.
+#ifndef QSA_DEC_NW_BF16
+#define QSA_DEC_NW_BF16 12
+#endif
+#ifndef QSA_DEC_NS_BF16
+#define QSA_DEC_NS_BF16 2
+#endif
 template <int D, int NT, bool FP8>
 struct DecodeShape {
-  static constexpr int NW = (!FP8 && NT <= 2) ? 12 : 8;
-  static constexpr int NS = (!FP8 && NT <= 2) ? 2 : (FP8 ? 4 : 3);
+  static constexpr int NW = (!FP8 && NT <= 2) ? QSA_DEC_NW_BF16 : 8;
+  static constexpr int NS = (!FP8 && NT <= 2) ? QSA_DEC_NS_BF16 : (FP8 ? 4 : 3);
 };
 
 template <int D, int NT, bool FP8>
