@@ -403,7 +403,7 @@ struct ItemWalker {
 };
 
 #ifndef QSA_SCAN_MIN_CTAS
-#define QSA_SCAN_MIN_CTAS 6
+#define QSA_SCAN_MIN_CTAS 5
 #endif
 #ifndef QSA_SCAN_LOAD
 #define QSA_SCAN_LOAD 2
@@ -443,7 +443,9 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   return pol;
 }
 
-template <int DI>
+// BPPC: micro-blocks per page when it is a compile-time constant (16 for
+// 64-token pages, 4 for 16-token pages), 0 for any page size.
+template <int DI, int BPPC>
 __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_kernel(Params p) {
   constexpr int kLPR = DI / 8;                    // lanes per row (16 B each)
   constexpr int kRPI = 32 / kLPR;                 // rows per load instruction
@@ -496,9 +498,37 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
       q0 = qq.x;
       q1 = qq.y;
     }
+    uint4 v[kItemLoads];
+    constexpr int kB = BPPC > 0 ? BPPC : 1;  // keeps the constant arithmetic defined
+    constexpr bool kFixed = BPPC > 0 && (kB % kRPI == 0) &&
+                            (kRowsPerItem % kB == 0 || kB % kRowsPerItem == 0);
+    if (kFixed && row0 + kRowsPerItem <= n) {
+      // whole item inside the request, page geometry known at compile time:
+      // one page base per page of the item, constant offsets per load; an
+      // invalid page reads page 0 instead (scores garbage, error recorded)
+      constexpr int kPagesPerItem = kRowsPerItem >= kB ? kRowsPerItem / kB : 1;
+      const int16_t *base[kPagesPerItem];
+#pragma unroll
+      for (int q = 0; q < kPagesPerItem; ++q) {
+        const int j = (row0 + q * kB) / kB - lp0;  // 0 .. kPagesPerItem-1 here
+        int pg = __shfl_sync(0xffffffffu, pg_lane, j & 31);
+        if (pg < 0) {
+          if (lane == 0) record_error(kErrBounds);
+          pg = 0;
+        }
+        base[q] = p.c.kc + ((long long)pg * kB + (kRowsPerItem >= kB ? 0 : row0 % kB)) * DI;
+      }
+#pragma unroll
+      for (int i = 0; i < kItemLoads; ++i) {
+        const int rr = i * kRPI;  // row of load i (before row_in) within the item
+        const int q = kRowsPerItem >= kB ? rr / kB : 0;
+        const int rin = kRowsPerItem >= kB ? rr % kB : rr;
+        v[i] = scan_load(reinterpret_cast<const uint4 *>(base[q] + (rin + row_in) * DI + sub * 8),
+                         pol_stream);
+      }
+    } else {
     // issue this item's loads; the lane's row advances by kRPI per load, so
     // its (logical page, row in page) pair is stepped instead of divided
-    uint4 v[kItemLoads];
     int lp = (row0 + row_in) / bpp;
     int off = (row0 + row_in) - lp * bpp;
 #pragma unroll
@@ -525,6 +555,7 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
         off -= bpp;
         ++lp;
       }
+    }
     }
     // prefetch the next item's block-table entries
     it += nwarps;

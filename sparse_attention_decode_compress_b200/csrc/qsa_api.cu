@@ -100,12 +100,12 @@ size_t select_smem() { return sizeof(qsa::topk::SelSmem) + 128; }
 
 // Scan (persistent grid, scores to the buffer) then selection (one CTA per
 // request), back to back on the caller's stream.
-template <int DI>
+template <int DI, int BPPC>
 qsa_status launch_index_topk(const qsa::topk::Params &p, cudaStream_t stream) {
   using namespace qsa::topk;
   static bool done_sel[kMaxDevices] = {false};
   static int blocks_per_sm[kMaxDevices] = {0};
-  auto kernel = index_scan_kernel<DI>;
+  auto kernel = index_scan_kernel<DI, BPPC>;
   const int dev = current_device();
   {
     std::lock_guard<std::mutex> lk(g_mutex);
@@ -284,10 +284,14 @@ qsa_status qsa_index_topk(const qsa_cache *cache, int32_t B, const int8_t *q_idx
   p.scores = scores ? scores
                     : reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + kTicketBytes);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int P = cache->page_size;
   switch (cache->idx_dim) {
-    case 32: return launch_index_topk<32>(p, s);
-    case 64: return launch_index_topk<64>(p, s);
-    default: return launch_index_topk<128>(p, s);
+    case 32: return P == 64 ? launch_index_topk<32, 16>(p, s)
+                  : P == 16 ? launch_index_topk<32, 4>(p, s) : launch_index_topk<32, 0>(p, s);
+    case 64: return P == 64 ? launch_index_topk<64, 16>(p, s)
+                  : P == 16 ? launch_index_topk<64, 4>(p, s) : launch_index_topk<64, 0>(p, s);
+    default: return P == 64 ? launch_index_topk<128, 16>(p, s)
+                  : P == 16 ? launch_index_topk<128, 4>(p, s) : launch_index_topk<128, 0>(p, s);
   }
 }
 
