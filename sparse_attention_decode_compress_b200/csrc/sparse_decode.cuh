@@ -94,25 +94,34 @@ __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl) {
   __syncwarp();
   int nvalid = 0, last = -1;
   const int n_entries = (L > 0) ? p.topk : 0;
-  for (int k = lane; k < n_entries; k += 32) {
-    const int v = sel_r[k];
-    const bool valid = v >= 0;
-    nvalid += __popc(__ballot_sync(__activemask(), valid));
-    if (valid) {
-      last = max(last, v);
-      const long long t = 4LL * v;
-      int lo = 0, hi = p.S;  // split s with tb[s] <= t < tb[s+1]
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (pl.tb[mid] <= t) lo = mid; else hi = mid;
+  constexpr int kBatch = 16;  // entries per lane loaded before any is used
+  for (int base = 0; base < n_entries; base += 32 * kBatch) {
+    int v[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int k = base + j * 32 + lane;
+      v[j] = (k < n_entries) ? sel_r[k] : -1;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const bool valid = v[j] >= 0;
+      nvalid += valid;
+      if (valid) {
+        last = max(last, v[j]);
+        const long long t = 4LL * v[j];
+        int lo = 0, hi = p.S;  // split s with tb[s] <= t < tb[s+1]
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (pl.tb[mid] <= t) lo = mid; else hi = mid;
+        }
+        atomicAdd(&pl.cnt[lo], 1);
       }
-      atomicAdd(&pl.cnt[lo], 1);
     }
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) {
     last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
-    nvalid = max(nvalid, __shfl_xor_sync(0xffffffffu, nvalid, o));
+    nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
   }
   __syncwarp();
   if (lane == 0) {
