@@ -127,8 +127,11 @@ qsa_status launch_index_topk(const qsa::topk::Params &p, cudaStream_t stream) {
 }
 
 // ---------------------------------------------------------------- decode --
+// Chunks of one (request, kv head): every split contributes at most one
+// partial chunk beyond ceil(extended entries / chunk), and the extended list
+// holds at most topk + 2 entries.
 int decode_chunk_slots(int topk, int S) {
-  return (topk + 2 + qsa::dec::kChunkBlocks - 1) / qsa::dec::kChunkBlocks + S;
+  return (topk + 2 + qsa::dec::kChunkBlocks - 1) / qsa::dec::kChunkBlocks + S - 1;
 }
 
 // Worker warps per SM and ring depth of the tensor-core decode kernel: as

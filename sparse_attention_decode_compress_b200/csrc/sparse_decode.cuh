@@ -29,7 +29,10 @@ namespace dec {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kChunkBlocks = 64;
+#ifndef QSA_CHUNK_BLOCKS
+#define QSA_CHUNK_BLOCKS 64
+#endif
+constexpr int kChunkBlocks = QSA_CHUNK_BLOCKS;  // micro-blocks per work item
 constexpr int kChunkTokens = kChunkBlocks * 4;  // 256
 constexpr int kStageTokens = 64;
 constexpr int kStagesPerChunk = kChunkTokens / kStageTokens;  // 4
@@ -67,7 +70,6 @@ struct Plan {
   int e_bound[kMaxSplits + 1];
   int ch_count[kMaxSplits];
   long long tb[kMaxSplits + 1];  // token boundary of each split
-  int cnt[kMaxSplits];           // selected blocks per split
 };
 
 // Entry k of the extended selection of request r.
@@ -75,11 +77,13 @@ __device__ __forceinline__ int ext_block(const int32_t *sel_r, const Plan &pl, i
   return k < pl.nvalid ? sel_r[k] : pl.extra[k - pl.nvalid];
 }
 
-// One warp reads the selection row once, coalesced, and counts the selected
-// blocks of every split (split of a block: binary search of its first token
-// in the split boundaries); the list is ascending, so the running counts are
-// the split boundaries in the extended list.
-__device__ void make_plan(const Params &p, int r, int chunk, Plan &pl) {
+// One warp reads the selection row once, coalesced, and derives the split
+// boundaries in the extended list: the split index of a selected block
+// (binary search of its first token in the split boundaries) never
+// decreases along the ascending row, so the lane holding entry k writes
+// e_bound[s] = k for every split s it starts.  If `stash` is not NULL the row
+// is also copied there (entries [0, topk)).
+__device__ void make_plan(const Params &p, int r, int chunk, Plan &pl, int *stash = nullptr) {
   const int lane = threadIdx.x & 31;
   const int32_t *sel_r = p.sel + (long long)r * p.topk;
   int L = p.ctx_lens[r];
@@ -90,7 +94,10 @@ __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl) {
   const int p0 = L - p.T;
   const long long NP = ((long long)L + p.c.page_size - 1) / p.c.page_size;
   if (lane <= p.S) pl.tb[lane] = min(((long long)lane * NP / p.S) * p.c.page_size, (long long)L);
-  if (lane < p.S) pl.cnt[lane] = 0;
+  __syncwarp();
+  // below[s] (kept in e_bound[s] by lane 0): selected blocks starting
+  // before the token boundary of split s
+  if (lane < p.S) pl.e_bound[lane] = 0;
   __syncwarp();
   int nvalid = 0, last = -1;
   const int n_entries = (L > 0) ? p.topk : 0;
@@ -104,18 +111,18 @@ __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl) {
     }
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
-      const bool valid = v[j] >= 0;
-      nvalid += valid;
-      if (valid) {
-        last = max(last, v[j]);
-        const long long t = 4LL * v[j];
-        int lo = 0, hi = p.S;  // split s with tb[s] <= t < tb[s+1]
-        while (hi - lo > 1) {
-          const int mid = (lo + hi) >> 1;
-          if (pl.tb[mid] <= t) lo = mid; else hi = mid;
-        }
-        atomicAdd(&pl.cnt[lo], 1);
-      }
+      const int k = base + j * 32 + lane;
+      if (stash && k < n_entries) stash[k] = v[j];
+      nvalid += v[j] >= 0;
+      last = max(last, v[j]);
+    }
+#pragma unroll 1
+    for (int sb = 1; sb < p.S; ++sb) {
+      const long long tbs = pl.tb[sb];
+      int cnt = 0;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) cnt += __popc(__ballot_sync(0xffffffffu, v[j] >= 0 && 4LL * v[j] < tbs));
+      if (lane == 0) pl.e_bound[sb] += cnt;
     }
   }
 #pragma unroll
@@ -137,15 +144,17 @@ __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl) {
     }
     pl.n_extra = ne;
     pl.nE = nvalid + ne;
+    // speculative-tail blocks follow every selected block: they move the
+    // boundaries of the splits after theirs
+    pl.e_bound[0] = 0;
+    for (int s = 1; s < p.S; ++s) {
+      int add = 0;
+      for (int x = 0; x < ne; ++x) add += (4LL * pl.extra[x] < pl.tb[s]);
+      pl.e_bound[s] = min(pl.e_bound[s], nvalid) + add;
+    }
+    pl.e_bound[p.S] = pl.nE;
     int cum = 0;
     pl.active = 0;
-    pl.e_bound[0] = 0;
-    for (int s = 0; s < p.S; ++s) {
-      int n = pl.cnt[s];
-      for (int x = 0; x < ne; ++x)
-        n += (4LL * pl.extra[x] >= pl.tb[s] && 4LL * pl.extra[x] < pl.tb[s + 1]);
-      pl.e_bound[s + 1] = pl.e_bound[s] + n;
-    }
     for (int s = 0; s < p.S; ++s) {
       const int n = pl.e_bound[s + 1] - pl.e_bound[s];
       const int ch = (n + kChunkBlocks - 1) / kChunkBlocks;

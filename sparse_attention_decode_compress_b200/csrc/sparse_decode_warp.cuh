@@ -64,46 +64,61 @@ __device__ void write_empty_splits_warp(const Params &p, const Plan &pl, int r, 
 // Token i is visible to query token t (position p_t = p0 + t) when i <= p_t
 // and (its block is selected or i > p0).
 template <typename WS, bool FP8>
-__device__ void fill_meta_warp(const Params &p, const Plan &pl, int r, int g, WS &W, int lane) {
-  const int32_t *sel_r = p.sel + (long long)r * p.topk;
+__device__ void fill_meta_warp(const Params &p, const Plan &pl, int r, int g, WS &W, int lane,
+                               const int *stash) {
+  const int32_t *sel_r = stash ? stash : p.sel + (long long)r * p.topk;
   const int P = p.c.page_size, Hkv = p.c.num_kv_heads;
-  int bl[kChunkTokens / 32];
+  const bool pow2 = (P & (P - 1)) == 0;
+  const int lgP = 31 - __clz(P);
+  // one lane per micro-block (kChunkBlocks / 32 each): one page lookup per
+  // block, four token rows
+  constexpr int kPer = kChunkBlocks / 32;
+  int bl[kPer], pg[kPer];
 #pragma unroll
-  for (int i = 0; i < kChunkTokens / 32; ++i) {
-    const int k = lane + 32 * i;
-    const int e = pl.e_begin + k / 4;
+  for (int i = 0; i < kPer; ++i) {
+    const int e = pl.e_begin + lane + 32 * i;
     bl[i] = (e < pl.e_end) ? ext_block(sel_r, pl, e) : -1;
   }
 #pragma unroll
-  for (int i = 0; i < kChunkTokens / 32; ++i) {
-    const int k = lane + 32 * i;
-    const int b = bl[i];
-    int off = -1;
-    unsigned vm = 0;
-    float ks = 1.f, vs = 1.f;
-    if (b >= 0) {
-      const long long t = 4LL * b + (k & 3);
-      if (t < pl.L) {
-        const int page = physical_page(p.c, r, t / P);
-        if (page >= 0) {
-          off = (int)(((long long)page * P + (t % P)) * Hkv + g);
-          const bool ins = (pl.e_begin + k / 4) < pl.nvalid;
-          for (int q = 0; q < p.T; ++q)
-            if (t <= (long long)pl.p0 + q && (ins || t > pl.p0)) vm |= 1u << q;
-          if (FP8) {
-            ks = p.c.k_scale[(long long)page * Hkv + g];
-            vs = p.c.v_scale[(long long)page * Hkv + g];
-          }
-        }
-      } else if ((k & 3) == 0 && 4LL * b >= pl.L) {
+  for (int i = 0; i < kPer; ++i) {
+    pg[i] = -1;
+    if (bl[i] >= 0) {
+      const long long t0 = 4LL * bl[i];
+      if (t0 < pl.L) {
+        pg[i] = physical_page(p.c, r, pow2 ? (t0 >> lgP) : t0 / P);
+      } else {
         record_error(kErrBadInput);  // selected block beyond the context
       }
     }
-    W.off[k] = off;
-    W.vmask[k] = (unsigned char)vm;
-    if (FP8) {
-      W.ks[k] = ks;
-      W.vs[k] = vs;
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = pl.e_begin + lane + 32 * i;
+    const int b = bl[i];
+    const bool ins = e < pl.nvalid;
+    float ks = 1.f, vs = 1.f;
+    if (FP8 && pg[i] >= 0) {
+      ks = p.c.k_scale[(long long)pg[i] * Hkv + g];
+      vs = p.c.v_scale[(long long)pg[i] * Hkv + g];
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int k = 4 * (lane + 32 * i) + j;  // chunk token index
+      const long long t = 4LL * b + j;
+      int off = -1;
+      unsigned vm = 0;
+      if (pg[i] >= 0 && t < pl.L) {
+        const long long tin = pow2 ? (t & (P - 1)) : t % P;
+        off = (int)(((long long)pg[i] * P + tin) * Hkv + g);
+        for (int q = 0; q < p.T; ++q)
+          if (t <= (long long)pl.p0 + q && (ins || t > pl.p0)) vm |= 1u << q;
+      }
+      W.off[k] = off;
+      W.vmask[k] = (unsigned char)vm;
+      if (FP8) {
+        W.ks[k] = ks;
+        W.vs[k] = vs;
+      }
     }
   }
 }
@@ -186,14 +201,10 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p
     const int c = it % p.nch;
     const int g = (it / p.nch) % Hkv;
     const int r = it / (p.nch * Hkv);
-    make_plan(p, r, c, pl);
-    __syncwarp();
-    if (c == 0) write_empty_splits_warp<D>(p, pl, r, g, lane);
-    if (!pl.active) continue;
-    fill_meta_warp<WS, FP8>(p, pl, r, g, W, lane);
 
     // Q as B fragments: n-tile j, k-step kk: b0 = Q[row 8j+gq][16kk+2cq, +1],
-    // b1 = Q[row 8j+gq][16kk+2cq+8, +9]; rows >= M are zero
+    // b1 = Q[row 8j+gq][16kk+2cq+8, +9]; rows >= M are zero.  Issued first so
+    // the loads overlap the plan.
     uint32_t qb[NT][MD][2];
     {
       const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
@@ -210,6 +221,15 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p
         }
       }
     }
+    // the selection row goes to the last ring slot (idle until stage NS-1)
+    constexpr int kStashInts = (int)(sizeof(W.ring[0]) / sizeof(int));
+    int *stash = p.topk <= kStashInts ? reinterpret_cast<int *>(&W.ring[NS - 1][0][0]) : nullptr;
+    make_plan(p, r, c, pl, stash);
+    __syncwarp();
+    if (c == 0) write_empty_splits_warp<D>(p, pl, r, g, lane);
+    if (!pl.active) continue;
+    fill_meta_warp<WS, FP8>(p, pl, r, g, W, lane, stash);
+
     // query token of each of this lane's columns (rows 8j + 2cq + e); -1 = padding
     int tcol[NT][2];
 #pragma unroll
