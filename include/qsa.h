@@ -216,6 +216,33 @@ qsa_status qsa_lse_merge(int32_t num_splits, int64_t rows, int32_t D, const floa
                          const float *lse_part, float *o, float *lse, qsa_stream_t stream);
 
 /*
+ * qsa_index_topk_noalloc — qsa_index_topk without a caller workspace.
+ *
+ * The source pages have no counterpart to this entry point; it exists for
+ * callers that cannot hand the library device memory of their own: code that
+ * runs where cudaMalloc is not allowed or not wanted (inside a plugin of a
+ * framework that owns all allocations, or on a latency-critical path where an
+ * allocation would synchronise the device), and that therefore cannot
+ * provide the score workspace.
+ *
+ * Same arguments and results as qsa_index_topk (sel only; no score output).
+ * The scores go to a fixed array compiled into libqsa.so: 8,388,608 int32
+ * (32 MiB), held on every GPU that loads the library until the process
+ * exits.  Calls with B * max_blocks above that are rejected with
+ * QSA_ERR_UNSUPPORTED before anything is launched.  Nothing is allocated:
+ * the first call on a device looks up the array's device address (with
+ * that device current) and keeps it, so make that first call before any
+ * stream capture.  All calls share the array: calls that overlap on the GPU
+ * (two streams, or two devices' threads racing on the same device) race on
+ * it; calls in order on one stream do not.  QSA_ERR_CUDA if the address
+ * lookup fails.
+ */
+qsa_status qsa_index_topk_noalloc(const qsa_cache *cache, int32_t B, const int8_t *q_idx,
+                                  const int32_t *ctx_lens, const int32_t *n_sel,
+                                  int32_t max_blocks, int32_t topk, int32_t *sel,
+                                  qsa_stream_t stream);
+
+/*
  * qsa_get_device_error — synchronise `stream`, then read and clear the
  * current device's error word.  Returns QSA_OK when no kernel recorded a
  * problem, else the first recorded code (QSA_ERR_BOUNDS, QSA_ERR_TIMEOUT,

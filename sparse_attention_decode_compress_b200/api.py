@@ -147,6 +147,27 @@ def qsa_index_topk(cache: QSACache, q_idx: torch.Tensor, ctx_lens: torch.Tensor,
                               _stream(stream)), "qsa_index_topk")
 
 
+def qsa_index_topk_noalloc(cache: QSACache, q_idx: torch.Tensor, ctx_lens: torch.Tensor,
+                           n_sel: torch.Tensor | None, max_blocks: int, topk: int,
+                           sel: torch.Tensor, stream=None) -> None:
+    """qsa_index_topk for callers that cannot provide a workspace: the
+    scores live in a fixed 32 MiB array inside libqsa.so (B * max_blocks
+    must not exceed 8,388,608)."""
+    _need(q_idx, torch.int8, "q_idx")
+    _need(ctx_lens, torch.int32, "ctx_lens")
+    _need(sel, torch.int32, "sel")
+    B = q_idx.shape[0]
+    if sel.shape != (B, topk):
+        raise ValueError("sel must be [B, topk]")
+    if n_sel is not None:
+        _need(n_sel, torch.int32, "n_sel")
+    s = cache.struct()
+    lib = _lib.load()
+    _check(lib.qsa_index_topk_noalloc(ctypes.byref(s), B, _ptr(q_idx), _ptr(ctx_lens), _ptr(n_sel),
+                                      int(max_blocks), int(topk), _ptr(sel), _stream(stream)),
+           "qsa_index_topk_noalloc")
+
+
 def qsa_sparse_decode(cache: QSACache, q: torch.Tensor, ctx_lens: torch.Tensor,
                       sel: torch.Tensor, sm_scale: float, num_splits: int,
                       o_part: torch.Tensor, lse_part: torch.Tensor, workspace: torch.Tensor,

@@ -410,3 +410,82 @@ qsa_status qsa_get_device_error(qsa_stream_t stream, uint32_t *flags_out) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// qsa_index_topk_noalloc: qsa_index_topk for callers that cannot allocate.
+//
+// The score buffer of this variant is a fixed array in the library's device
+// image: every GPU that loads libqsa.so holds kNoAllocScoreInts int32 (32 MiB)
+// for it until the process exits.  Host code only ever sees a host-side
+// stand-in for that array's name, so its device address is looked up once
+// per device (cudaGetSymbolAddress, with that device current) and passed to
+// the kernels.  Every call shares the array; the scan writes every score a
+// selection then reads, so nothing in it needs clearing between calls, and
+// calls that overlap on the GPU race on it.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr long long kNoAllocScoreInts = 8LL * 1024 * 1024;  // B * max_blocks limit
+static __device__ __align__(256) int32_t g_noalloc_scores[kNoAllocScoreInts];
+
+int32_t *g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the score array on the current device (set-up on first
+// use per device); NULL if the runtime could not provide it.
+int32_t *noalloc_scores_ptr() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scores) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = static_cast<int32_t *>(ptr);
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+qsa_status qsa_index_topk_noalloc(const qsa_cache *cache, int32_t B, const int8_t *q_idx,
+                                  const int32_t *ctx_lens, const int32_t *n_sel,
+                                  int32_t max_blocks, int32_t topk, int32_t *sel,
+                                  qsa_stream_t stream) {
+  qsa_status st = check_cache(cache);
+  if (st != QSA_OK) return st;
+  if (B < 0) return QSA_ERR_INVALID_ARG;
+  if (topk < 1 || topk > qsa::topk::kMaxTopk) return QSA_ERR_INVALID_ARG;
+  if (max_blocks < 1 || max_blocks > (1 << 24)) return QSA_ERR_INVALID_ARG;
+  if ((long long)B * max_blocks > kNoAllocScoreInts) return QSA_ERR_UNSUPPORTED;
+  if (B == 0) return QSA_OK;
+  if (!q_idx || !ctx_lens || !sel || !cache->kc) return QSA_ERR_INVALID_ARG;
+  if (cache->idx_dim != 32 && cache->idx_dim != 64 && cache->idx_dim != 128)
+    return QSA_ERR_UNSUPPORTED;
+  if (!aligned(cache->kc, 16) || !aligned(q_idx, 4)) return QSA_ERR_INVALID_ARG;
+  int32_t *scores = noalloc_scores_ptr();
+  if (!scores) return QSA_ERR_CUDA;
+
+  qsa::topk::Params p;
+  p.c = to_dev(cache);
+  p.B = B;
+  p.q_idx = q_idx;
+  p.ctx_lens = ctx_lens;
+  p.n_sel = n_sel;
+  p.max_blocks = max_blocks;
+  p.topk = topk;
+  p.sel = sel;
+  p.scores = scores;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int P = cache->page_size;
+  switch (cache->idx_dim) {
+    case 32: return P == 64 ? launch_index_topk<32, 16>(p, s)
+                  : P == 16 ? launch_index_topk<32, 4>(p, s) : launch_index_topk<32, 0>(p, s);
+    case 64: return P == 64 ? launch_index_topk<64, 16>(p, s)
+                  : P == 16 ? launch_index_topk<64, 4>(p, s) : launch_index_topk<64, 0>(p, s);
+    default: return P == 64 ? launch_index_topk<128, 16>(p, s)
+                  : P == 16 ? launch_index_topk<128, 4>(p, s) : launch_index_topk<128, 0>(p, s);
+  }
+}
+
+}  // extern "C"
