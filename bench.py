@@ -48,6 +48,31 @@ def parse_args(argv=None):
 
 
 # ---------------------------------------------------------------------------
+# Multi-rank helpers (one process per GPU; replicas of the workload)
+# ---------------------------------------------------------------------------
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch (independent replicas, weak scaling)."""
+    return base_seed + rank
+
+
+def max_over_ranks(value_ms: float, world: int, device=None) -> float:
+    """The slowest rank's time (every rank calls this, in the same order)."""
+    if world <= 1:
+        return value_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_rate(per_rank_units: int, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: units of all ranks over the slowest rank's time."""
+    return world * per_rank_units * steps / (ms_max / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # Algorithmic bytes (what the method must move), per query and per launch
 # ---------------------------------------------------------------------------
 
@@ -268,7 +293,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         from dataclasses import replace
         w = replace(w, batch=args.batch)
     S = args.splits
-    batch = make_batch(w, dev, seed=w.seed + rank)
+    batch = make_batch(w, dev, seed=rank_seed(w.seed, rank))
     B, T = w.batch, w.T
     L_host = batch.ctx_lens_host
     max_blocks = int((L_host.max() + 3) // 4)
@@ -343,10 +368,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     st, flags = qsa_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error in the timed region: status {st} flags {flags}")
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
 
     # ---- end to end through the C ABI with host buffers
     e2e = None
@@ -388,12 +410,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * B * T * Ke / (e_ms / 1e3), "unit": UNIT,
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": weak_scaling_rate(B * T, world, Ke, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     clocks = sampler.stop() if rank == 0 else None
@@ -405,7 +423,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     tot_bytes = sum(a["total"] for a in ab)
     peaks = measured_peaks()
     queries_per_step = B * T
-    value = world * queries_per_step * K / (ms / 1e3)
+    value = weak_scaling_rate(queries_per_step, world, K, ms)
     hbm = (tot_bytes * K / (ms / 1e3)) / 1e9
     achieved = idx_bytes / (topk_ms / 1e3) / 1e9
     line = {
