@@ -106,6 +106,23 @@ def algorithmic_bytes(w, L: int, num_splits: int) -> dict:
                 total=idx + dec + merge + append)
 
 
+def index_topk_traffic(batch: int):
+    """DRAM bytes of one qsa_index_topk launch from the committed ncu capture
+    (profiles/roofline_traffic.json), scaled by requests; None when the
+    kernel source changed since the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        t = json.load(f)
+    with open(os.path.join(ROOT, t["source"]), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if not sha.startswith(t["source_sha256_prefix"]):
+        return None
+    return int(t["dram_bytes_per_request"]) * batch
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -441,7 +458,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "hbm_pct_of_nominal_8tbs": round(100 * hbm / 8000.0, 2),
         "roofline": {"bound": "hbm", "kernel": "index_topk", "achieved": round(achieved, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "peak_source": peaks["source"], "traffic": None,
+                     "peak_source": peaks["source"], "traffic": index_topk_traffic(B),
                      "launch_ms": round(topk_ms, 5), "algorithmic_bytes_per_launch": idx_bytes},
         "kernel_ms": {"index_topk": round(topk_ms, 5), "sparse_decode": round(dec_ms, 5)},
         "gpu_launches": QSADecodeStep.KERNELS_PER_STEP * K,
