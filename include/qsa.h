@@ -189,10 +189,13 @@ size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32
  *   o_part   [S, B, T, Hq, D] float32 output
  *   lse_part [S, B, T, Hq] float32 output (natural log)
  *   workspace  >= qsa_sparse_decode_workspace_bytes(...), 16-byte aligned,
- *            ZERO-FILLED before first use, left zeroed by every completed
- *            call (same rule as qsa_index_topk).
- * Errors: QSA_ERR_INVALID_ARG / QSA_ERR_UNSUPPORTED on the host; page or
- * position violations -> QSA_ERR_BOUNDS on the device.
+ *            ZERO-FILLED before first use and left zeroed by every completed
+ *            call: its header holds the work counter and the per-split
+ *            tickets; the rest holds chunk partials.
+ * Errors: QSA_ERR_INVALID_ARG / QSA_ERR_UNSUPPORTED on the host
+ * (QSA_ERR_UNSUPPORTED also when num_pages * page_size * Hkv exceeds
+ * 2^31 - 1 cache rows); page or position violations -> QSA_ERR_BOUNDS on the
+ * device.
  */
 qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
                              const void *q, int32_t q_dtype, const int32_t *ctx_lens,

@@ -5,6 +5,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -127,11 +128,25 @@ qsa_status launch_index_topk(const qsa::topk::Params &p, cudaStream_t stream) {
 }
 
 // ---------------------------------------------------------------- decode --
-// Chunks of one (request, kv head): every split contributes at most one
-// partial chunk beyond ceil(extended entries / chunk), and the extended list
-// holds at most topk + 2 entries.
-int decode_chunk_slots(int topk, int S) {
-  return (topk + 2 + qsa::dec::kChunkBlocks - 1) / qsa::dec::kChunkBlocks + S - 1;
+// Chunk slots of one (request, kv head) for chunks of `chunk` micro-blocks:
+// a split of n entries takes ceil(n / chunk) chunks, so the splits together
+// take at most ceil(E / chunk) + S - 1, and the extended list holds at most
+// E = topk + 2 entries.
+int decode_chunk_slots(int topk, int S, int chunk) {
+  return (topk + 2 + chunk - 1) / chunk + S - 1;
+}
+
+// Chunk size of the persistent decode: the largest work items that still
+// give every worker warp at most one of them (one wave, no tail of second
+// items), within [kMinChunkBlocks, kChunkBlocks].  A batch with more
+// (request, kv head) pairs than warps takes the largest chunks.
+int decode_chunk_blocks(int B, int Hkv, int topk, int S, long long workers) {
+  const long long pairs = (long long)B * Hkv;
+  const long long per_pair = workers / (pairs > 0 ? pairs : 1);
+  const long long n_chunks = per_pair - (S - 1);
+  int chunk = qsa::dec::kChunkBlocks;
+  if (n_chunks > 0) chunk = (int)std::min<long long>(chunk, (topk + 2 + n_chunks - 1) / n_chunks);
+  return std::max(chunk, qsa::dec::kMinChunkBlocks);
 }
 
 // Worker warps per SM and ring depth of the tensor-core decode kernel: as
@@ -150,7 +165,7 @@ struct DecodeShape {
 };
 
 template <int D, int NT, bool FP8>
-qsa_status launch_decode_warp(const qsa::dec::Params &p, cudaStream_t stream) {
+qsa_status launch_decode_warp(qsa::dec::Params p, cudaStream_t stream) {
   constexpr int NW = DecodeShape<D, NT, FP8>::NW;
   constexpr int NS = DecodeShape<D, NT, FP8>::NS;
   static bool done[kMaxDevices] = {false};
@@ -169,13 +184,19 @@ qsa_status launch_decode_warp(const qsa::dec::Params &p, cudaStream_t stream) {
     }
   }
   const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
-  kernel<<<bps * sm_count(dev), NW * 32, smem, stream>>>(p);
+  const int ctas = bps * sm_count(dev);
+  p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, (long long)ctas * NW);
+  p.nch = decode_chunk_slots(p.topk, p.S, p.chunk);
+  kernel<<<ctas, NW * 32, smem, stream>>>(p);
   return launch_status();
 }
 
 template <int D>
-qsa_status launch_decode_f32(const qsa::dec::Params &p, dim3 grid, cudaStream_t stream) {
+qsa_status launch_decode_f32(qsa::dec::Params p, cudaStream_t stream) {
   static bool done[kMaxDevices] = {false};
+  p.chunk = qsa::dec::kChunkBlocks;  // one CTA per chunk slot
+  p.nch = decode_chunk_slots(p.topk, p.S, p.chunk);
+  const dim3 grid((unsigned)p.nch, (unsigned)p.c.num_kv_heads, (unsigned)p.B);
   auto kernel = qsa::dec::sparse_decode_f32_kernel<D>;
   const size_t smem = sizeof(qsa::dec::F32Smem<D>) + 128;
   {
@@ -197,9 +218,8 @@ qsa_status dispatch_decode_nt(const qsa::dec::Params &p, int NT, cudaStream_t st
 }
 
 template <int D>
-qsa_status dispatch_decode_d(const qsa::dec::Params &p, int kv_dtype, dim3 grid,
-                             cudaStream_t stream) {
-  if (kv_dtype == QSA_F32) return launch_decode_f32<D>(p, grid, stream);
+qsa_status dispatch_decode_d(const qsa::dec::Params &p, int kv_dtype, cudaStream_t stream) {
+  if (kv_dtype == QSA_F32) return launch_decode_f32<D>(p, stream);
   const int NT = (p.M + 7) / 8;  // query rows on the N side, tiles of 8
   if (kv_dtype == QSA_FP8_E4M3) return dispatch_decode_nt<D, true>(p, NT, stream);
   return dispatch_decode_nt<D, false>(p, NT, stream);
@@ -302,7 +322,8 @@ size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32
                                          int32_t D, int32_t topk, int32_t num_splits) {
   if (B < 0 || T < 1 || Hq < 1 || Hkv < 1 || D < 1 || topk < 1 || num_splits < 1) return 0;
   const size_t M = (size_t)(Hq / Hkv) * T;
-  const size_t nch = decode_chunk_slots(topk, num_splits);
+  // room for the smallest chunks the launch may pick
+  const size_t nch = decode_chunk_slots(topk, num_splits, qsa::dec::kMinChunkBlocks);
   const size_t slots = (size_t)B * Hkv * nch;
   return kTicketBytes + align_up(slots * M * D * sizeof(float)) + align_up(slots * M * sizeof(float));
 }
@@ -332,6 +353,8 @@ qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32
   }
   if (B == 0) return QSA_OK;
   if (B > 65535 || Hkv > 65535) return QSA_ERR_UNSUPPORTED;
+  // cache rows are indexed with 32-bit integers
+  if ((long long)cache->num_pages * cache->page_size * Hkv > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
   if ((size_t)B * Hkv * num_splits * sizeof(int32_t) >
       kTicketBytes - qsa::dec::kCounterInts * sizeof(int32_t))
     return QSA_ERR_UNSUPPORTED;
@@ -346,7 +369,7 @@ qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32
   if (workspace_bytes < qsa_sparse_decode_workspace_bytes(B, T, Hq, Hkv, D, topk, num_splits))
     return QSA_ERR_INVALID_ARG;
 
-  const int nch = decode_chunk_slots(topk, num_splits);
+  const int nch = decode_chunk_slots(topk, num_splits, qsa::dec::kMinChunkBlocks);
   const int M = G * T;
   qsa::dec::Params p;
   p.c = to_dev(cache);
@@ -369,11 +392,11 @@ qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32
   const size_t slots = (size_t)B * Hkv * nch;
   p.ws_o = reinterpret_cast<float *>(ws + kTicketBytes);
   p.ws_lse = reinterpret_cast<float *>(ws + kTicketBytes + align_up(slots * M * D * sizeof(float)));
-  p.nch = nch;
-  const dim3 grid((unsigned)nch, (unsigned)Hkv, (unsigned)B);
+  p.nch = nch;  // the launch sets nch and chunk for its kernel
+  p.chunk = qsa::dec::kMinChunkBlocks;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (D == 64) return dispatch_decode_d<64>(p, cache->kv_dtype, grid, s);
-  return dispatch_decode_d<128>(p, cache->kv_dtype, grid, s);
+  if (D == 64) return dispatch_decode_d<64>(p, cache->kv_dtype, s);
+  return dispatch_decode_d<128>(p, cache->kv_dtype, s);
 }
 
 qsa_status qsa_lse_merge(int32_t num_splits, int64_t rows, int32_t D, const float *o_part,

@@ -12,7 +12,9 @@
 // kv head g, chunk).  The "extended selection" of r is the sorted selection
 // row followed by the speculative-tail blocks that are not selected; split s
 // owns the entries whose block lies in its page slice (a contiguous range,
-// since the list is sorted), cut into chunks of 64 micro-blocks (256 tokens).
+// since the list is sorted), cut into ceil(n / chunk) chunks of equal size
+// (to one entry), `chunk` <= kChunkBlocks micro-blocks being chosen by the
+// host for the batch shape.
 // A split with one chunk writes o_part/lse_part directly; a split with
 // several chunks stages them in the workspace and the chunk that finishes
 // last (atomic ticket) merges them by log-sum-exp.
@@ -30,12 +32,11 @@ namespace dec {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 #ifndef QSA_CHUNK_BLOCKS
-#define QSA_CHUNK_BLOCKS 64
+#define QSA_CHUNK_BLOCKS 128
 #endif
-constexpr int kChunkBlocks = QSA_CHUNK_BLOCKS;  // micro-blocks per work item
-constexpr int kChunkTokens = kChunkBlocks * 4;  // 256
-constexpr int kStageTokens = 64;
-constexpr int kStagesPerChunk = kChunkTokens / kStageTokens;  // 4
+constexpr int kChunkBlocks = QSA_CHUNK_BLOCKS;  // capacity of a work item, micro-blocks
+constexpr int kChunkTokens = kChunkBlocks * 4;
+constexpr int kMinChunkBlocks = 32;  // smallest chunk the host picks
 constexpr int kMaxSplits = 16;
 constexpr int kMaxT = 4;
 constexpr int kMaxRows = 32;  // G * T
@@ -58,6 +59,7 @@ struct Params {
   int32_t *tickets;  // [B, Hkv, S]
   int32_t *counters; // work counters of the persistent kernel (zero between calls)
   int nch;           // chunk slots per (r, g)
+  int chunk;         // target micro-blocks per chunk, kMinChunkBlocks..kChunkBlocks
 };
 
 // Per-CTA plan, computed by warp 0.
@@ -157,16 +159,17 @@ __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl, int *stas
     pl.active = 0;
     for (int s = 0; s < p.S; ++s) {
       const int n = pl.e_bound[s + 1] - pl.e_bound[s];
-      const int ch = (n + kChunkBlocks - 1) / kChunkBlocks;
+      const int ch = (n + p.chunk - 1) / p.chunk;  // chunks of n / ch <= p.chunk entries
       pl.ch_count[s] = ch;
       if (!pl.active && chunk >= cum && chunk < cum + ch) {
+        const int k = chunk - cum;
         pl.active = 1;
         pl.split = s;
         pl.nchunks_split = ch;
-        pl.chunk_in_split = chunk - cum;
+        pl.chunk_in_split = k;
         pl.first_chunk_of_split = cum;
-        pl.e_begin = pl.e_bound[s] + (chunk - cum) * kChunkBlocks;
-        pl.e_end = min(pl.e_bound[s + 1], pl.e_begin + kChunkBlocks);
+        pl.e_begin = pl.e_bound[s] + (int)((long long)k * n / ch);
+        pl.e_end = pl.e_bound[s] + (int)((long long)(k + 1) * n / ch);
       }
       cum += ch;
     }
@@ -361,7 +364,7 @@ struct F32Smem {
   Plan pl;
   float o[kMaxRows * D];
   float lse[kMaxRows];
-  float scratch[kMaxRows * (4096 / kChunkBlocks + 2 + kMaxSplits)];
+  float scratch[kMaxRows * (4096 / kChunkBlocks + 2 + kMaxSplits)];  // chunk = kChunkBlocks
   int flag;
 };
 

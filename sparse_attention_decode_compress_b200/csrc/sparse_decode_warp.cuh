@@ -29,11 +29,16 @@ struct WarpState {
   static constexpr int kRowBytes = D * (FP8 ? 1 : 2);
   alignas(128) uint8_t ring[NS][2][kTokW * kRowBytes];
   alignas(128) uint8_t cvt[FP8 ? 2 : 1][FP8 ? kTokW * D * 2 : 16];
-  int off[kChunkTokens];             // (token, head) row index in the cache, -1 = nothing to load
-  unsigned char vmask[kChunkTokens]; // bit t: the token is visible to query token t
-  float ks[FP8 ? kChunkTokens : 1];
-  float vs[FP8 ? kChunkTokens : 1];
+  int boff[kChunkBlocks];  // cache row (token, head g) of each micro-block's first token
+  // byte j of word b: visibility bits of token j of micro-block b (bit t:
+  // visible to query token t); a token visible to none is not loaded
+  uint32_t vmask4[kChunkBlocks];
+  float ks[FP8 ? kChunkBlocks : 1];  // fp8 scales of each micro-block's page
+  float vs[FP8 ? kChunkBlocks : 1];
   Plan pl;
+  __device__ __forceinline__ unsigned vmask(int tok) const {
+    return reinterpret_cast<const unsigned char *>(vmask4)[tok];
+  }
 };
 
 template <int D, bool FP8, int NW, int NS>
@@ -60,9 +65,11 @@ __device__ void write_empty_splits_warp(const Params &p, const Plan &pl, int r, 
   }
 }
 
-// Token metadata of the chunk: cache row, visibility bits and fp8 scales.
-// Token i is visible to query token t (position p_t = p0 + t) when i <= p_t
-// and (its block is selected or i > p0).
+// Micro-block metadata of the chunk: cache row of the first token, the
+// tokens' visibility bits and fp8 scales.  Token i is visible to query token
+// t (position p_t = p0 + t) when i <= p_t and (its block is selected or
+// i > p0).  A micro-block never straddles a page (P % 4 == 0), so token j of
+// block b sits j * Hkv rows after its first token.
 template <typename WS, bool FP8>
 __device__ void fill_meta_warp(const Params &p, const Plan &pl, int r, int g, WS &W, int lane,
                                const int *stash) {
@@ -70,8 +77,8 @@ __device__ void fill_meta_warp(const Params &p, const Plan &pl, int r, int g, WS
   const int P = p.c.page_size, Hkv = p.c.num_kv_heads;
   const bool pow2 = (P & (P - 1)) == 0;
   const int lgP = 31 - __clz(P);
-  // one lane per micro-block (kChunkBlocks / 32 each): one page lookup per
-  // block, four token rows
+  // one lane per micro-block (kChunkBlocks / 32 each), one page lookup per
+  // block; every block slot is written (slots past the chunk: nothing visible)
   constexpr int kPer = kChunkBlocks / 32;
   int bl[kPer], pg[kPer];
 #pragma unroll
@@ -93,32 +100,35 @@ __device__ void fill_meta_warp(const Params &p, const Plan &pl, int r, int g, WS
   }
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
-    const int e = pl.e_begin + lane + 32 * i;
-    const int b = bl[i];
+    const int kb = lane + 32 * i;  // chunk block index
+    const int e = pl.e_begin + kb;
+    const long long t0 = 4LL * bl[i];
     const bool ins = e < pl.nvalid;
+    int boff = -1;
+    uint32_t vm4 = 0;
     float ks = 1.f, vs = 1.f;
-    if (FP8 && pg[i] >= 0) {
-      ks = p.c.k_scale[(long long)pg[i] * Hkv + g];
-      vs = p.c.v_scale[(long long)pg[i] * Hkv + g];
-    }
+    if (pg[i] >= 0) {
+      const long long tin = pow2 ? (t0 & (P - 1)) : t0 % P;
+      boff = (int)(((long long)pg[i] * P + tin) * Hkv + g);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int k = 4 * (lane + 32 * i) + j;  // chunk token index
-      const long long t = 4LL * b + j;
-      int off = -1;
-      unsigned vm = 0;
-      if (pg[i] >= 0 && t < pl.L) {
-        const long long tin = pow2 ? (t & (P - 1)) : t % P;
-        off = (int)(((long long)pg[i] * P + tin) * Hkv + g);
-        for (int q = 0; q < p.T; ++q)
-          if (t <= (long long)pl.p0 + q && (ins || t > pl.p0)) vm |= 1u << q;
+      for (int j = 0; j < 4; ++j) {
+        const long long t = t0 + j;
+        unsigned vm = 0;
+        if (t < pl.L)
+          for (int q = 0; q < p.T; ++q)
+            if (t <= (long long)pl.p0 + q && (ins || t > pl.p0)) vm |= 1u << q;
+        vm4 |= vm << (8 * j);
       }
-      W.off[k] = off;
-      W.vmask[k] = (unsigned char)vm;
       if (FP8) {
-        W.ks[k] = ks;
-        W.vs[k] = vs;
+        ks = p.c.k_scale[(long long)pg[i] * Hkv + g];
+        vs = p.c.v_scale[(long long)pg[i] * Hkv + g];
       }
+    }
+    W.boff[kb] = boff;
+    W.vmask4[kb] = vm4;
+    if (FP8) {
+      W.ks[kb] = ks;
+      W.vs[kb] = vs;
     }
   }
 }
@@ -133,16 +143,19 @@ __device__ __forceinline__ void issue_stage_warp(const Params &p, WS &W, int slo
   constexpr int kItems = 2 * kTokW * kCh;
   const uint8_t *kbase = static_cast<const uint8_t *>(p.c.k_cache);
   const uint8_t *vbase = static_cast<const uint8_t *>(p.c.v_cache);
+  const int Hkv = p.c.num_kv_heads;
 #pragma unroll
   for (int i = 0; i < kItems / 32; ++i) {
     const int it = lane + 32 * i;
     const int kv = it / (kTokW * kCh);
     const int rem = it % (kTokW * kCh);
     const int row = rem / kCh, ch = rem % kCh;
-    const int off = W.off[st * kTokW + row];
+    const int tok = st * kTokW + row;
+    const bool load = W.vmask(tok) != 0u;
+    const int off = load ? W.boff[tok >> 2] + (tok & 3) * Hkv : 0;
     uint8_t *dst = W.ring[slot][kv] + (FP8 ? (row * kRowBytes + ch * 16) : swz<D>(row, ch));
-    const uint8_t *src = (kv ? vbase : kbase) + (long long)max(off, 0) * kRowBytes + ch * 16;
-    cp_async16_zfill(dst, src, off >= 0);
+    const uint8_t *src = (kv ? vbase : kbase) + (long long)off * kRowBytes + ch * 16;
+    cp_async16_zfill(dst, src, load);
   }
 }
 
@@ -307,13 +320,13 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p
         for (int e = 0; e < 4; ++e) sacc[j][e] += sac2[j][e];
 
       // ---- mask, online softmax per column, P^T as bf16 hi + lo B fragments
-      const unsigned vm0 = W.vmask[tb + gq], vm1 = W.vmask[tb + gq + 8];
+      const unsigned vm0 = W.vmask(tb + gq), vm1 = W.vmask(tb + gq + 8);
       float ksc0 = 1.f, ksc1 = 1.f, vsc0 = 1.f, vsc1 = 1.f;
       if constexpr (FP8) {
-        ksc0 = W.ks[tb + gq];
-        ksc1 = W.ks[tb + gq + 8];
-        vsc0 = W.vs[tb + gq];
-        vsc1 = W.vs[tb + gq + 8];
+        ksc0 = W.ks[(tb + gq) >> 2];
+        ksc1 = W.ks[(tb + gq + 8) >> 2];
+        vsc0 = W.vs[(tb + gq) >> 2];
+        vsc1 = W.vs[(tb + gq + 8) >> 2];
       }
       uint32_t bhi[NT][2], blo[NT][2];
       bool rescale = false;

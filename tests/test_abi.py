@@ -45,9 +45,10 @@ def test_workspace_sizes():
     tick = 64 * 1024
     assert lib.qsa_index_topk_workspace_bytes(128, 65536) == tick + 128 * 65536 * 4
     assert lib.qsa_index_topk_workspace_bytes(-1, 3) == 0
-    # decode: B*Hkv*nch slots of (M*D floats + M floats), nch = ceil((topk+2)/64) + S - 1
+    # decode: B*Hkv*nch slots of (M*D floats + M floats), nch = ceil((topk+2)/32) + S - 1
+    # (room for the smallest chunks, 32 micro-blocks, a launch may pick)
     B, T, Hq, Hkv, D, K, S = 128, 1, 16, 2, 128, 512, 2
-    nch = -(-(K + 2) // 64) + S - 1
+    nch = -(-(K + 2) // 32) + S - 1
     M = Hq // Hkv * T
     def al(x):
         return -(-x // 256) * 256
