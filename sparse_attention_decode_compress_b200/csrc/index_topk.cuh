@@ -11,25 +11,33 @@
 // (256 B per block at d = 128).  Persistent warps walk 8 KiB items (request,
 // run of rows), load them with 16-byte streaming loads (16 per lane in
 // flight), turn them into scores with dp2a (int16 x int8 pairs) and a
-// butterfly reduce-scatter, and write the scores to an L2-resident buffer.  A second kernel selects, one CTA per
-// request: a 4096-bin histogram of the high score bits finds the threshold
-// bin, the blocks above it are kept outright, the threshold bin's blocks are
-// gathered in shared memory and bitonic-sorted by (score desc, index asc),
-// and the kept indices are bitonic-sorted ascending.  A request whose
-// threshold bin overflows shared memory falls back to exact radix passes
-// over its scores.  (Selecting inside the scan kernel, in the CTA that
+// butterfly reduce-scatter, and write the scores to an L2-resident buffer.
+// A second kernel selects, one CTA per request: a 4096-bin histogram of the
+// high score bits finds the threshold bin, the blocks above it are kept
+// outright, the threshold bin's blocks are gathered in shared memory and
+// ranked by (score desc, index asc) by counting.  Kept blocks are marked in
+// a shared bitmap that a prefix sum of popcounts reads out in ascending
+// order.  A request whose threshold bin overflows shared memory falls back
+// to exact radix passes over its scores.  (Selecting inside the scan kernel, in the CTA that
 // finished a request last, serialised the selections: that CTA fell behind
 // and kept finishing last.)
 #pragma once
+#include <climits>
+
 #include "qsa_common.cuh"
 
 namespace qsa {
 namespace topk {
 
-constexpr int kHistBins = 4096;  // first digit: bits [25:14] of score + 2^25
+// Scores are ordered through 25-bit keys, score + 2^24: |score| <= 2^23 for
+// d <= 128 and int8 inputs.  The first digit is key bits [24:12] (8192 bins
+// of 4096 score units); the exact fallback resolves bits [11:6] and [5:0].
+constexpr int kScoreBias = 1 << 24;
+constexpr int kDigit1Shift = 12;
+constexpr int kHistBins = 1 << 13;
+constexpr int kFbDigitBits = 6;
 constexpr int kCandCap = 2048;   // threshold-bin candidates kept in shared memory
 constexpr int kMaxTopk = 4096;
-constexpr int kScoreBias = 1 << 25;  // |score| <= 2^23 for d <= 128 and int8 inputs
 
 struct Params {
   CacheDev c;
@@ -58,7 +66,7 @@ __device__ __forceinline__ int request_blocks(const Params &p, int r, bool repor
   return (int)n;
 }
 
-// Order-preserving unsigned key of a score in [0, 2^26).  Valid inputs give
+// Order-preserving unsigned key of a score in [0, 2^25).  Valid inputs give
 // |score| <= 2^23; the clamp only keeps corrupt cache contents from indexing
 // outside the histogram.
 __device__ __forceinline__ uint32_t score_key(int s) {
@@ -73,13 +81,74 @@ __device__ __forceinline__ uint32_t score_key(int s) {
 
 constexpr int kSelThreads = 1024;
 constexpr int kSelBatch = 8;  // int4 loads in flight per thread
+constexpr int kBitmapWords = 8192;  // requests of <= 262,144 blocks mark kept blocks in a bitmap
+#ifndef QSA_SEL_MATCH
+#define QSA_SEL_MATCH 0
+#endif
 
 struct SelSmem {
   int hist[kHistBins];  // also the kept-index list (kMaxTopk ints) after pass A
   unsigned long long cand[kCandCap];
+  uint32_t bits[kBitmapWords];  // bit i: block i kept
   int warp_tot[kSelThreads / 32];
   int bin, above, nkeep, ncand, fb_key, fb_above, fb_idx;
 };
+
+// Exclusive prefix sum of one int per thread over the CTA (uses
+// sm.warp_tot; begins and ends with a barrier).
+__device__ __forceinline__ int block_exclusive_sum(int v, SelSmem &sm, int tid) {
+  const int lane = tid & 31, w = tid >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  __syncthreads();
+  if (lane == 31) sm.warp_tot[w] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int i = 0; i < w; ++i) base += sm.warp_tot[i];
+  return base + incl - v;
+}
+
+// Appends index i to sm.cand (key x) for the lanes with `take` set: one
+// shared atomic per warp instead of one per lane.
+__device__ __forceinline__ void append_cand(bool take, unsigned long long x, SelSmem &sm) {
+  const unsigned am = __activemask();
+  const unsigned bal = __ballot_sync(am, take);
+  if (bal == 0u) return;
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(bal) - 1;
+  int base = 0;
+  if (lane == leader) base = atomicAdd(&sm.ncand, __popc(bal));
+  base = __shfl_sync(am, base, leader);
+  if (take) {
+    const int slot = base + __popc(bal & ((1u << lane) - 1u));
+    if (slot < kCandCap) sm.cand[slot] = x;
+  }
+}
+
+// Writes the set bits of bits[0 .. ceil(n/32)) as ascending indices:
+// exactly K bits are set.
+__device__ void write_from_bits(const uint32_t *bits, int n, int K, int32_t *out, SelSmem &sm,
+                                int tid) {
+  const int W = (n + 31) >> 5;
+  const int per = (W + kSelThreads - 1) / kSelThreads;
+  const int w0 = min(W, tid * per), w1 = min(W, w0 + per);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
+  int pos = block_exclusive_sum(cnt, sm, tid);
+  for (int w = w0; w < w1; ++w) {
+    uint32_t m = bits[w];
+    while (m) {
+      const int b = __ffs(m) - 1;
+      m &= m - 1u;
+      if (pos < K) out[pos] = w * 32 + b;
+      ++pos;
+    }
+  }
+}
 
 __device__ __forceinline__ void bitonic_sort_i32(int *a, int n_pow2, int tid) {
   for (int k = 2; k <= n_pow2; k <<= 1) {
@@ -106,11 +175,12 @@ __device__ __forceinline__ int next_pow2(int x) {
   return p;
 }
 
-// Applies f(index, score) to every score of a row, reading it with batched
-// 16-byte loads from its first 16-byte boundary (rows are 4-byte aligned;
-// the row stride need not be a multiple of 4).
-template <typename F>
-__device__ __forceinline__ void for_each_score(const int32_t *sc, int n, int tid, F f) {
+// Reads every score of a row with batched 16-byte loads from its first
+// 16-byte boundary (rows are 4-byte aligned; the row stride need not be a
+// multiple of 4): fq(index, int4) for each aligned quad, f(index, score) for
+// the scores before and after them.
+template <typename FQ, typename F>
+__device__ __forceinline__ void for_each_score_q(const int32_t *sc, int n, int tid, FQ fq, F f) {
   const int head = min(n, (int)(((16u - (uint32_t)(reinterpret_cast<uintptr_t>(sc) & 15u)) & 15u) >> 2));
   if (tid < head) f(tid, __ldcg(sc + tid));
   const int4 *v4 = reinterpret_cast<const int4 *>(sc + head);
@@ -125,16 +195,63 @@ __device__ __forceinline__ void for_each_score(const int32_t *sc, int n, int tid
 #pragma unroll
     for (int j = 0; j < kSelBatch; ++j) {
       const int i = base + j * kSelThreads + tid;
-      if (i < nv) {
-        const int e = head + 4 * i;
-        f(e, v[j].x);
-        f(e + 1, v[j].y);
-        f(e + 2, v[j].z);
-        f(e + 3, v[j].w);
-      }
+      if (i < nv) fq(head + 4 * i, v[j]);
     }
   }
   for (int i = head + 4 * nv + tid; i < n; i += kSelThreads) f(i, __ldcg(sc + i));
+}
+
+// Visits the scores of a row that may pass a filter: quads are loaded in
+// batches, reduced to one bit each by keep4(int4), and only the (rare)
+// flagged quads are read again and handed to f(index, score) element by
+// element; the scores before and after the aligned quads always go to f.
+template <typename K4, typename F>
+__device__ __forceinline__ void for_each_flagged_score(const int32_t *sc, int n, int tid, K4 keep4,
+                                                       F f) {
+  const int head = min(n, (int)(((16u - (uint32_t)(reinterpret_cast<uintptr_t>(sc) & 15u)) & 15u) >> 2));
+  if (tid < head) f(tid, __ldcg(sc + tid));
+  const int4 *v4 = reinterpret_cast<const int4 *>(sc + head);
+  const int nv = (n - head) >> 2;
+  for (int base = 0; base < nv; base += kSelThreads * kSelBatch) {
+    int4 v[kSelBatch];
+#pragma unroll
+    for (int j = 0; j < kSelBatch; ++j) {
+      const int i = base + j * kSelThreads + tid;
+      v[j] = (i < nv) ? __ldcg(v4 + i) : make_int4(INT_MIN, INT_MIN, INT_MIN, INT_MIN);
+    }
+    unsigned flags = 0;
+#pragma unroll
+    for (int j = 0; j < kSelBatch; ++j) {
+      const int i = base + j * kSelThreads + tid;
+      flags |= (i < nv && keep4(v[j]) ? 1u : 0u) << j;
+    }
+    while (flags) {
+      const int j = __ffs(flags) - 1;
+      flags &= flags - 1u;
+      const int i = base + j * kSelThreads + tid;
+      const int4 w = __ldcg(v4 + i);
+      const int e = head + 4 * i;
+      f(e, w.x);
+      f(e + 1, w.y);
+      f(e + 2, w.z);
+      f(e + 3, w.w);
+    }
+  }
+  for (int i = head + 4 * nv + tid; i < n; i += kSelThreads) f(i, __ldcg(sc + i));
+}
+
+// Applies f(index, score) to every score of a row.
+template <typename F>
+__device__ __forceinline__ void for_each_score(const int32_t *sc, int n, int tid, F f) {
+  for_each_score_q(
+      sc, n, tid,
+      [&](int e, int4 v) {
+        f(e, v.x);
+        f(e + 1, v.y);
+        f(e + 2, v.z);
+        f(e + 3, v.w);
+      },
+      f);
 }
 
 // Finds, in hist[0..nbins), the bin where the running count taken from the
@@ -178,21 +295,22 @@ __device__ void find_rank_bin_desc(const int *hist, int rank, SelSmem &sm, int t
 // then the kept set is gathered.
 __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, int tid) {
   int *hist = sm.hist;
+  constexpr int kFbBins = 1 << kFbDigitBits;
   uint32_t prefix = (uint32_t)sm.bin;  // key >> shift
   int above = sm.above;
-  int shift = 14;
+  int shift = kDigit1Shift;
   for (int pass = 0; pass < 2; ++pass) {
-    const int nshift = shift - 7;
+    const int nshift = shift - kFbDigitBits;
     for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
     __syncthreads();
     for_each_score(sc, n, tid, [&](int, int s) {
       const uint32_t k = score_key(s);
-      if ((k >> shift) == prefix) atomicAdd(&hist[(k >> nshift) & 127], 1);
+      if ((k >> shift) == prefix) atomicAdd(&hist[(k >> nshift) & (kFbBins - 1)], 1);
     });
     __syncthreads();
     if (tid == 0) {
       int cum = above;
-      for (int b = 127; b >= 0; --b) {
+      for (int b = kFbBins - 1; b >= 0; --b) {
         if (cum + hist[b] >= K) {
           sm.fb_key = b;
           sm.fb_above = cum;
@@ -202,7 +320,7 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
       }
     }
     __syncthreads();
-    prefix = (prefix << 7) | (uint32_t)sm.fb_key;
+    prefix = (prefix << kFbDigitBits) | (uint32_t)sm.fb_key;
     above = sm.fb_above;
     shift = nshift;
   }
@@ -292,31 +410,53 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
     return;
   }
   int *hist = sm.hist;
+  // kept blocks go to a bitmap when the request fits it, else to a list
+  const bool use_bits = n <= kBitmapWords * 32;
+  const int nwords = use_bits ? (n + 31) >> 5 : 0;
   // pass A: histogram of the first digit (bits [25:14] of the key)
   for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
-  __syncthreads();
-  for_each_score(sc, n, tid, [&](int, int s) { atomicAdd(&hist[score_key(s) >> 14], 1); });
-  __syncthreads();
-  find_rank_bin_desc(hist, K, sm, tid);
-  const uint32_t b1 = (uint32_t)sm.bin;
-  // pass B: keep the blocks above the threshold bin, gather the bin's blocks
-  int *keep = sm.hist;
+  for (int i = tid; i < nwords; i += kSelThreads) sm.bits[i] = 0u;
   if (tid == 0) {
     sm.nkeep = 0;
     sm.ncand = 0;
   }
   __syncthreads();
-  for_each_score(sc, n, tid, [&](int i, int s) {
-    const uint32_t k = score_key(s);
-    const uint32_t d1 = k >> 14;
-    if (d1 > b1) {
-      const int slot = atomicAdd(&sm.nkeep, 1);
-      if (slot < kMaxTopk) keep[slot] = i;
-    } else if (d1 == b1) {
-      const int slot = atomicAdd(&sm.ncand, 1);
-      if (slot < kCandCap) sm.cand[slot] = ((unsigned long long)(0xffffffffu - k) << 32) | (uint32_t)i;
-    }
+  for_each_score(sc, n, tid, [&](int, int s) {
+    const int b = (int)(score_key(s) >> kDigit1Shift);
+#if QSA_SEL_MATCH
+    const unsigned am = __activemask();
+    const unsigned peers = __match_any_sync(am, b);
+    if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[b], __popc(peers));
+#else
+    atomicAdd(&hist[b], 1);
+#endif
   });
+  __syncthreads();
+  find_rank_bin_desc(hist, K, sm, tid);
+  const uint32_t b1 = (uint32_t)sm.bin;
+  // pass B: keep the blocks above the threshold bin, gather the bin's
+  // blocks; a quad whose largest score is below the bin is skipped whole
+  int *keep = sm.hist;
+  auto visit = [&](int i, int s) {
+    const uint32_t k = score_key(s);
+    const uint32_t d1 = k >> kDigit1Shift;
+    if (d1 > b1) {
+      if (use_bits) {
+        atomicOr(&sm.bits[i >> 5], 1u << (i & 31));
+      } else {
+        const int slot = atomicAdd(&sm.nkeep, 1);
+        if (slot < kMaxTopk) keep[slot] = i;
+      }
+    }
+    append_cand(d1 == b1, ((unsigned long long)(0xffffffffu - k) << 32) | (uint32_t)i, sm);
+  };
+  for_each_flagged_score(
+      sc, n, tid,
+      [&](int4 v) {
+        const int m = max(max(v.x, v.y), max(v.z, v.w));
+        return (score_key(m) >> kDigit1Shift) >= b1;
+      },
+      visit);
   __syncthreads();
   const int above = sm.above;
   const int ncand = sm.ncand;
@@ -329,13 +469,24 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
       const unsigned long long x = sm.cand[i];
       int rank = 0;
       for (int j = 0; j < ncand; ++j) rank += (sm.cand[j] < x);
-      if (rank < need) keep[above + rank] = (int)(uint32_t)(x & 0xffffffffu);
+      if (rank < need) {
+        const int idx = (int)(uint32_t)(x & 0xffffffffu);
+        if (use_bits) atomicOr(&sm.bits[idx >> 5], 1u << (idx & 31));
+        else keep[above + rank] = idx;
+      }
     }
     __syncthreads();
   } else {
-    select_fallback(sc, n, K, sm, tid);
+    select_fallback(sc, n, K, sm, tid);  // the kept list, in sm.hist
+    if (use_bits) {
+      for (int i = tid; i < nwords; i += kSelThreads) sm.bits[i] = 0u;
+      __syncthreads();
+      for (int i = tid; i < K; i += kSelThreads) atomicOr(&sm.bits[keep[i] >> 5], 1u << (keep[i] & 31));
+      __syncthreads();
+    }
   }
-  write_ascending(keep, K, out, sm, tid);
+  if (use_bits) write_from_bits(sm.bits, n, K, out, sm, tid);
+  else write_ascending(keep, K, out, sm, tid);
 }
 
 // ------------------------------------------------------------- the scan --

@@ -99,6 +99,30 @@ def test_two_valued_keys_many_ties():
     _check_all(b, step, cache, 2)
 
 
+def test_extreme_scores_order_exactly():
+    """Scores at the ends of the int8 range: q = -128 everywhere and 700
+    blocks of keys -128 score exactly 2^23 (tied), 300 more score 2^23 - 128,
+    the rest mix -128 / 127 / -127.  The selection's ordering keys must span
+    the whole score range."""
+    w = replace(WORKLOADS["b32_32k"], planted=0)
+    b = make_batch(w, "cuda", ctx_lens=[32768, 12000], seed=13)
+    g = torch.Generator(device="cuda").manual_seed(2)
+    pick = torch.randint(0, 3, b.k_idx.shape, generator=g, device="cuda")
+    vals = torch.tensor([-128, 127, -127], dtype=torch.int8, device="cuda")
+    b.k_idx.copy_(vals[pick])
+    blocks = torch.randperm(32768 // 4, generator=torch.Generator().manual_seed(3))[:1000]
+    for j, blk in enumerate(blocks.tolist()):
+        rows = b.k_idx[4 * blk:4 * blk + 4]
+        rows.fill_(-128)
+        if j >= 700:
+            rows[0, 0] = -127
+    b.q_idx.fill_(-128)
+    step, cache = H.run_gpu(b, 2)
+    top = sorted(blocks[:700].tolist())[:512]
+    assert step.sel[0].cpu().tolist() == top
+    _check_all(b, step, cache, 2)
+
+
 def test_split_count_invariance():
     w = WORKLOADS["b128_256k"]
     b = make_batch(w, "cuda", ctx_lens=[40000, 30001], seed=21)
