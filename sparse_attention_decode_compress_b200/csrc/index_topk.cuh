@@ -82,17 +82,27 @@ __device__ __forceinline__ uint32_t score_key(int s) {
 constexpr int kSelThreads = 1024;
 constexpr int kSelBatch = 8;  // int4 loads in flight per thread
 constexpr int kBitmapWords = 8192;  // requests of <= 262,144 blocks mark kept blocks in a bitmap
-#ifndef QSA_SEL_MATCH
-#define QSA_SEL_MATCH 0
-#endif
 
 struct SelSmem {
-  int hist[kHistBins];  // also the kept-index list (kMaxTopk ints) after pass A
+  int hist[kHistBins];  // also the kept-index list (kMaxTopk ints) on the list path
   unsigned long long cand[kCandCap];
   uint32_t bits[kBitmapWords];  // bit i: block i kept
   int warp_tot[kSelThreads / 32];
   int bin, above, nkeep, ncand, fb_key, fb_above, fb_idx;
 };
+
+// Sum of the per-warp totals sm.warp_tot[0 .. w) (all 32 written before a
+// barrier), by a shuffle scan in every warp.
+__device__ __forceinline__ int warps_before(const SelSmem &sm, int w, int lane) {
+  int x = sm.warp_tot[lane];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  const int before = __shfl_sync(0xffffffffu, x, (w + 31) & 31);
+  return w == 0 ? 0 : before;
+}
 
 // Exclusive prefix sum of one int per thread over the CTA (uses
 // sm.warp_tot; begins and ends with a barrier).
@@ -107,9 +117,7 @@ __device__ __forceinline__ int block_exclusive_sum(int v, SelSmem &sm, int tid) 
   __syncthreads();
   if (lane == 31) sm.warp_tot[w] = incl;
   __syncthreads();
-  int base = 0;
-  for (int i = 0; i < w; ++i) base += sm.warp_tot[i];
-  return base + incl - v;
+  return warps_before(sm, w, lane) + incl - v;
 }
 
 // Appends index i to sm.cand (key x) for the lanes with `take` set: one
@@ -271,9 +279,7 @@ __device__ void find_rank_bin_desc(const int *hist, int rank, SelSmem &sm, int t
   }
   if (lane == 31) sm.warp_tot[w] = incl;
   __syncthreads();
-  int base = 0;
-  for (int i = 0; i < w; ++i) base += sm.warp_tot[i];
-  const int excl = base + incl - local;
+  const int excl = warps_before(sm, w, lane) + incl - local;
   if (excl < rank && rank <= excl + local) {
     int cum = excl;
     for (int k = 0; k < per; ++k) {
@@ -395,8 +401,46 @@ __device__ void write_ascending(int *keep, int K, int32_t *out, SelSmem &sm, int
   for (int i = tid; i < K; i += kSelThreads) out[i] = keep[i];
 }
 
+// The two passes of the selection over a score row: a histogram of the
+// first digit, then a pass that keeps the blocks above the threshold bin
+// (bitmap when use_bits, else the list in sm.hist) and gathers the bin's
+// blocks.
+__device__ void select_passes(const int32_t *sc, int n, int K, bool use_bits, SelSmem &sm,
+                               int tid) {
+  for_each_score(sc, n, tid, [&](int, int sv) {
+    atomicAdd(&sm.hist[score_key(sv) >> kDigit1Shift], 1);
+  });
+  __syncthreads();
+  find_rank_bin_desc(sm.hist, K, sm, tid);
+  const uint32_t b1 = (uint32_t)sm.bin;
+  int *keep = sm.hist;
+  auto visit = [&](int i, int sv) {
+    const uint32_t k = score_key(sv);
+    const uint32_t d1 = k >> kDigit1Shift;
+    if (d1 > b1) {
+      if (use_bits) {
+        atomicOr(&sm.bits[i >> 5], 1u << (i & 31));
+      } else {
+        const int slot = atomicAdd(&sm.nkeep, 1);
+        if (slot < kMaxTopk) keep[slot] = i;
+      }
+    }
+    append_cand(d1 == b1, ((unsigned long long)(0xffffffffu - k) << 32) | (uint32_t)i, sm);
+  };
+  // a quad whose largest score is below the threshold bin is skipped whole
+  for_each_flagged_score(
+      sc, n, tid,
+      [&](int4 v) {
+        const int m = max(max(v.x, v.y), max(v.z, v.w));
+        return (score_key(m) >> kDigit1Shift) >= b1;
+      },
+      visit);
+  __syncthreads();
+}
+
 // Selection kernel: grid = B, one request per CTA.
 __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
+  pdl_open();
   extern __shared__ uint8_t smem_raw[];
   SelSmem &sm = *reinterpret_cast<SelSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int r = blockIdx.x;
@@ -409,55 +453,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
     for (int i = tid; i < K; i += kSelThreads) out[i] = i < n ? i : -1;
     return;
   }
-  int *hist = sm.hist;
   // kept blocks go to a bitmap when the request fits it, else to a list
   const bool use_bits = n <= kBitmapWords * 32;
   const int nwords = use_bits ? (n + 31) >> 5 : 0;
-  // pass A: histogram of the first digit (bits [25:14] of the key)
-  for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+  for (int i = tid; i < kHistBins; i += kSelThreads) sm.hist[i] = 0;
   for (int i = tid; i < nwords; i += kSelThreads) sm.bits[i] = 0u;
   if (tid == 0) {
     sm.nkeep = 0;
     sm.ncand = 0;
   }
   __syncthreads();
-  for_each_score(sc, n, tid, [&](int, int s) {
-    const int b = (int)(score_key(s) >> kDigit1Shift);
-#if QSA_SEL_MATCH
-    const unsigned am = __activemask();
-    const unsigned peers = __match_any_sync(am, b);
-    if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[b], __popc(peers));
-#else
-    atomicAdd(&hist[b], 1);
-#endif
-  });
-  __syncthreads();
-  find_rank_bin_desc(hist, K, sm, tid);
-  const uint32_t b1 = (uint32_t)sm.bin;
-  // pass B: keep the blocks above the threshold bin, gather the bin's
-  // blocks; a quad whose largest score is below the bin is skipped whole
+  select_passes(sc, n, K, use_bits, sm, tid);
   int *keep = sm.hist;
-  auto visit = [&](int i, int s) {
-    const uint32_t k = score_key(s);
-    const uint32_t d1 = k >> kDigit1Shift;
-    if (d1 > b1) {
-      if (use_bits) {
-        atomicOr(&sm.bits[i >> 5], 1u << (i & 31));
-      } else {
-        const int slot = atomicAdd(&sm.nkeep, 1);
-        if (slot < kMaxTopk) keep[slot] = i;
-      }
-    }
-    append_cand(d1 == b1, ((unsigned long long)(0xffffffffu - k) << 32) | (uint32_t)i, sm);
-  };
-  for_each_flagged_score(
-      sc, n, tid,
-      [&](int4 v) {
-        const int m = max(max(v.x, v.y), max(v.z, v.w));
-        return (score_key(m) >> kDigit1Shift) >= b1;
-      },
-      visit);
-  __syncthreads();
   const int above = sm.above;
   const int ncand = sm.ncand;
   if (ncand <= kCandCap) {
@@ -598,6 +605,7 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
 // 64-token pages, 4 for 16-token pages), 0 for any page size.
 template <int DI, int BPPC>
 __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_kernel(Params p) {
+  pdl_open();
   constexpr int kLPR = DI / 8;                    // lanes per row (16 B each)
   constexpr int kRPI = 32 / kLPR;                 // rows per load instruction
   constexpr int kRowsPerItem = kItemLoads * kRPI; // 4096 / DI

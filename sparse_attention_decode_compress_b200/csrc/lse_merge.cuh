@@ -16,6 +16,7 @@ constexpr int kMergeMaxSplits = 64;
 __global__ void __launch_bounds__(kMergeThreads) lse_merge_kernel(
     int S, long long rows, int D, const float *__restrict__ o_part,
     const float *__restrict__ lse_part, float *__restrict__ o, float *__restrict__ lse) {
+  pdl_open();
   const long long row = (long long)blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;

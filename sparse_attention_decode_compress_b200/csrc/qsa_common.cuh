@@ -23,6 +23,20 @@ __device__ uint32_t g_error_flags;
 
 __device__ __forceinline__ void record_error(uint32_t bits) { atomicOr(&g_error_flags, bits); }
 
+// Programmatic dependent launch.  The library launches its kernels (all
+// but compress_append, see qsa_api.cu) with programmatic stream
+// serialisation: such a kernel may be
+// scheduled once every CTA of the kernel before it has started, so its
+// CTAs are resident, past their launch, when that kernel ends.  Every kernel
+// opens with pdl_open() before anything else: it lets the next kernel
+// launch, then waits until the work before it on the stream has completed
+// and its memory is visible.  Without a programmatic dependency (a kernel
+// from elsewhere, a copy) the wait returns at once.
+__device__ __forceinline__ void pdl_open() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // A bounded wait gives up after about this many SM cycles (~1 s at 1.9 GHz).
 constexpr long long kWaitCycles = 2000000000LL;
 

@@ -370,6 +370,7 @@ struct F32Smem {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) sparse_decode_f32_kernel(Params p) {
+  pdl_open();
   extern __shared__ uint8_t smem_raw[];
   using SM = F32Smem<D>;
   SM &sm = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));

@@ -194,6 +194,7 @@ __device__ __forceinline__ void convert_fp8_rows_warp(const uint8_t *raw, uint8_
 // tiles of 8, so G*T = 8 uses every MMA lane.
 template <int D, int NT, bool FP8, int NW, int NS>
 __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p) {
+  pdl_open();
   extern __shared__ uint8_t smem_raw[];
   using SM = WarpSmem<D, FP8, NW, NS>;
   using WS = WarpState<D, FP8, NS>;
