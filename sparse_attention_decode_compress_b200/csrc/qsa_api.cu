@@ -163,7 +163,10 @@ int decode_chunk_slots(int topk, int S, int chunk) {
 // Chunk size of the persistent decode: the largest work items that still
 // give every worker warp at most one of them (one wave, no tail of second
 // items), within [kMinChunkBlocks, kChunkBlocks].  A batch with more
-// (request, kv head) pairs than warps takes the largest chunks.
+// (request, kv head) pairs than warps takes the largest chunks.  (Two or
+// three smaller chunks per warp, balanced through the work counter,
+// measured ~30% slower: each chunk's fixed plan / metadata / epilogue
+// latency is paid again.)
 int decode_chunk_blocks(int B, int Hkv, int topk, int S, long long workers) {
   const long long pairs = (long long)B * Hkv;
   const long long per_pair = workers / (pairs > 0 ? pairs : 1);

@@ -88,6 +88,15 @@ __device__ __forceinline__ int ext_block(const int32_t *sel_r, const Plan &pl, i
 __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl, int *stash = nullptr) {
   const int lane = threadIdx.x & 31;
   const int32_t *sel_r = p.sel + (long long)r * p.topk;
+  constexpr int kBatch = 16;  // entries per lane loaded before any is used
+  // the first batch of the selection row is loaded together with the
+  // context length (the row is always readable; an empty context ignores it)
+  int v[kBatch];
+#pragma unroll
+  for (int j = 0; j < kBatch; ++j) {
+    const int k = j * 32 + lane;
+    v[j] = (k < p.topk) ? sel_r[k] : -1;
+  }
   int L = p.ctx_lens[r];
   if (L < p.T) {
     if (lane == 0) record_error(kErrBadInput);
@@ -103,13 +112,13 @@ __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl, int *stas
   __syncwarp();
   int nvalid = 0, last = -1;
   const int n_entries = (L > 0) ? p.topk : 0;
-  constexpr int kBatch = 16;  // entries per lane loaded before any is used
   for (int base = 0; base < n_entries; base += 32 * kBatch) {
-    int v[kBatch];
+    if (base > 0) {
 #pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
-      const int k = base + j * 32 + lane;
-      v[j] = (k < n_entries) ? sel_r[k] : -1;
+      for (int j = 0; j < kBatch; ++j) {
+        const int k = base + j * 32 + lane;
+        v[j] = (k < n_entries) ? sel_r[k] : -1;
+      }
     }
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {

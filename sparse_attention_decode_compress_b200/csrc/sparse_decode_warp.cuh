@@ -134,28 +134,37 @@ __device__ void fill_meta_warp(const Params &p, const Plan &pl, int r, int g, WS
 }
 
 // cp.async of stage st of the chunk into ring slot `slot` (rows swizzled for
-// bf16; fp8 rows land raw and are converted before use).
+// bf16; fp8 rows land raw and are converted before use).  A lane copies the
+// same 16-byte column of kTokW / kRowsPerPass rows of K and of V; their
+// metadata is read into registers before the first copy is issued.
 template <int D, bool FP8, typename WS>
 __device__ __forceinline__ void issue_stage_warp(const Params &p, WS &W, int slot, int st,
                                                  int lane) {
   constexpr int kRowBytes = WS::kRowBytes;
-  constexpr int kCh = kRowBytes / 16;  // 16-byte chunks per row
-  constexpr int kItems = 2 * kTokW * kCh;
+  constexpr int kCh = kRowBytes / 16;           // 16-byte chunks per row
+  constexpr int kRowsPerPass = 32 / kCh;        // rows one warp-wide pass covers
+  constexpr int kPasses = kTokW / kRowsPerPass;
   const uint8_t *kbase = static_cast<const uint8_t *>(p.c.k_cache);
   const uint8_t *vbase = static_cast<const uint8_t *>(p.c.v_cache);
   const int Hkv = p.c.num_kv_heads;
+  const int ch = lane % kCh, r0 = lane / kCh;
+  int off[kPasses];
+  bool load[kPasses];
 #pragma unroll
-  for (int i = 0; i < kItems / 32; ++i) {
-    const int it = lane + 32 * i;
-    const int kv = it / (kTokW * kCh);
-    const int rem = it % (kTokW * kCh);
-    const int row = rem / kCh, ch = rem % kCh;
-    const int tok = st * kTokW + row;
-    const bool load = W.vmask(tok) != 0u;
-    const int off = load ? W.boff[tok >> 2] + (tok & 3) * Hkv : 0;
-    uint8_t *dst = W.ring[slot][kv] + (FP8 ? (row * kRowBytes + ch * 16) : swz<D>(row, ch));
-    const uint8_t *src = (kv ? vbase : kbase) + (long long)off * kRowBytes + ch * 16;
-    cp_async16_zfill(dst, src, load);
+  for (int j = 0; j < kPasses; ++j) {
+    const int tok = st * kTokW + r0 + j * kRowsPerPass;
+    load[j] = W.vmask(tok) != 0u;
+    off[j] = load[j] ? W.boff[tok >> 2] + (tok & 3) * Hkv : 0;
+  }
+#pragma unroll
+  for (int kv = 0; kv < 2; ++kv) {
+#pragma unroll
+    for (int j = 0; j < kPasses; ++j) {
+      const int row = r0 + j * kRowsPerPass;
+      uint8_t *dst = W.ring[slot][kv] + (FP8 ? (row * kRowBytes + ch * 16) : swz<D>(row, ch));
+      const uint8_t *src = (kv ? vbase : kbase) + (long long)off[j] * kRowBytes + ch * 16;
+      cp_async16_zfill(dst, src, load[j]);
+    }
   }
 }
 
@@ -207,10 +216,19 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p
   const int gq = lane >> 2, cq = lane & 3;
   constexpr int MD = D / 16;  // m-tiles of O^T (16 dims each)
 
+  // first item: the warp's own index, numbered across CTAs first so that a
+  // batch with fewer items than warps still loads every SM evenly; later
+  // items: from the work counter, which hands out indices from the number
+  // of warps on
+  const int nwarps = gridDim.x * NW;
+  bool first = true;
   while (true) {
-    int it = 0;
-    if (lane == 0) it = atomicAdd(&p.counters[0], 1);
-    it = __shfl_sync(0xffffffffu, it, 0);
+    int it = warp * gridDim.x + blockIdx.x;
+    if (!first) {
+      if (lane == 0) it = nwarps + atomicAdd(&p.counters[0], 1);
+      it = __shfl_sync(0xffffffffu, it, 0);
+    }
+    first = false;
     if (it >= total_items) break;
     const int c = it % p.nch;
     const int g = (it / p.nch) % Hkv;
@@ -485,8 +503,7 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p
   }
   // every warp reports once; the last one resets the work counters
   if (lane == 0) {
-    const int total_warps = gridDim.x * NW;
-    if (atomicAdd(&p.counters[1], 1) == total_warps - 1) {
+    if (atomicAdd(&p.counters[1], 1) == nwarps - 1) {
       atomicExch(&p.counters[0], 0);
       atomicExch(&p.counters[1], 0);
     }
