@@ -155,6 +155,36 @@ qsa_status qsa_index_topk(const qsa_cache *cache, int32_t B, const int8_t *q_idx
                           int32_t topk, int32_t *sel, int32_t *scores, void *workspace,
                           size_t workspace_bytes, qsa_stream_t stream);
 
+/*
+ * qsa_index_topk_tokens — the selection as a token budget: fixed-width rows
+ * of request-relative token indices, padded with -1.
+ *
+ * Passage: PR #53896 report, QSAIndexer.forward excerpt (the indexer's
+ * budget is a token count, token_topk = indexer_budget; forward returns
+ * fixed-width request-relative token indices padded with -1; MTP step 0
+ * selects for the target row and later steps reuse it).
+ *
+ * Selects topk = budget / 4 micro-blocks exactly as qsa_index_topk does,
+ * then lists their tokens: with p0 = ctx_lens[r] - T (query token 0),
+ *   tokens[r][4k + j] = 4 b_k + j   if 4 b_k + j <= p0, else -1
+ * for the k-th kept block b_k in ascending order, and -1 in the groups of
+ * four past the kept blocks.  Only the block holding p0 can be cut, and it
+ * is the last kept one, so every row is ascending and its -1 sit at its end.
+ *
+ *   T        1 .. 4 query tokens per request (p0 as above)
+ *   budget   4 .. 16384, a multiple of 4 (the compress ratio)
+ *   tokens   [B, budget] int32 output, 16-byte aligned
+ *   sel      [B, budget / 4] int32 output of the kept blocks, or NULL
+ *   other arguments as for qsa_index_topk (topk = budget / 4)
+ * Errors: as qsa_index_topk; QSA_ERR_INVALID_ARG also for a budget that is
+ * not a positive multiple of 4, T out of range or a misaligned `tokens`.
+ */
+qsa_status qsa_index_topk_tokens(const qsa_cache *cache, int32_t B, const int8_t *q_idx,
+                                 const int32_t *ctx_lens, const int32_t *n_sel, int32_t T,
+                                 int32_t max_blocks, int32_t budget, int32_t *tokens,
+                                 int32_t *sel, int32_t *scores, void *workspace,
+                                 size_t workspace_bytes, qsa_stream_t stream);
+
 /* Workspace bytes qsa_sparse_decode needs. */
 size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32_t Hkv,
                                          int32_t D, int32_t topk, int32_t num_splits);

@@ -185,6 +185,22 @@ def selection_width(L: int, T: int) -> int:
 # Token sets and attention
 # ----------------------------------------------------------------------------
 
+def selection_tokens(sel: np.ndarray, L: int, T: int, budget: int) -> np.ndarray:
+    """The selection as a token budget: the tokens of the selected blocks
+    that query token 0 (position p0 = L - T) may see, i.e. positions <= p0,
+    ascending, padded with -1 to width `budget`.  [pr] QSAIndexer.forward
+    excerpt (the budget is a token count, token_topk = indexer_budget;
+    forward returns fixed-width request-relative token indices padded with
+    -1).  int32 [budget]."""
+    p0 = int(L) - int(T)
+    toks = sorted(4 * int(b) + j for b in np.asarray(sel) if b >= 0 for j in range(4)
+                  if 4 * int(b) + j <= p0)
+    out = np.full(int(budget), -1, dtype=np.int32)
+    k = min(len(toks), int(budget))
+    out[:k] = toks[:k]
+    return out
+
+
 def token_set(sel: np.ndarray, L: int, T: int, t: int) -> np.ndarray:
     """Token positions attended by query token t (position p_t = L - T + t).
 

@@ -43,6 +43,9 @@ SIGNATURES = {
     "qsa_index_topk_noalloc": (c_int32, [ctypes.POINTER(QsaCacheStruct), c_int32, c_void_p,
                                          c_void_p, c_void_p, c_int32, c_int32, c_void_p,
                                          c_void_p]),
+    "qsa_index_topk_tokens": (c_int32, [ctypes.POINTER(QsaCacheStruct), c_int32, c_void_p,
+                                        c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
+                                        c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "qsa_get_device_error": (c_int32, [c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
 }
 

@@ -168,6 +168,38 @@ def qsa_index_topk_noalloc(cache: QSACache, q_idx: torch.Tensor, ctx_lens: torch
            "qsa_index_topk_noalloc")
 
 
+def qsa_index_topk_tokens(cache: QSACache, q_idx: torch.Tensor, ctx_lens: torch.Tensor,
+                          n_sel: torch.Tensor | None, T: int, max_blocks: int, budget: int,
+                          tokens: torch.Tensor, sel: torch.Tensor | None,
+                          scores: torch.Tensor | None, workspace: torch.Tensor,
+                          stream=None) -> None:
+    """The selection as fixed-width rows of token indices ([B, budget],
+    -1 padded); `sel` ([B, budget // 4]) optionally receives the blocks."""
+    _need(q_idx, torch.int8, "q_idx")
+    _need(ctx_lens, torch.int32, "ctx_lens")
+    _need(tokens, torch.int32, "tokens")
+    B = q_idx.shape[0]
+    if tokens.shape != (B, budget):
+        raise ValueError("tokens must be [B, budget]")
+    if sel is not None:
+        _need(sel, torch.int32, "sel")
+        if sel.shape != (B, budget // 4):
+            raise ValueError("sel must be [B, budget // 4]")
+    if n_sel is not None:
+        _need(n_sel, torch.int32, "n_sel")
+    if scores is not None:
+        _need(scores, torch.int32, "scores")
+        if scores.shape != (B, max_blocks):
+            raise ValueError("scores must be [B, max_blocks]")
+    s = cache.struct()
+    lib = _lib.load()
+    _check(lib.qsa_index_topk_tokens(ctypes.byref(s), B, _ptr(q_idx), _ptr(ctx_lens), _ptr(n_sel),
+                                     int(T), int(max_blocks), int(budget), _ptr(tokens), _ptr(sel),
+                                     _ptr(scores), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "qsa_index_topk_tokens")
+
+
 def qsa_sparse_decode(cache: QSACache, q: torch.Tensor, ctx_lens: torch.Tensor,
                       sel: torch.Tensor, sm_scale: float, num_splits: int,
                       o_part: torch.Tensor, lse_part: torch.Tensor, workspace: torch.Tensor,

@@ -47,7 +47,9 @@ struct Params {
   const int32_t *n_sel;
   int max_blocks;
   int topk;
-  int32_t *sel;
+  int32_t *sel;      // [B, topk] kept block indices, or NULL
+  int32_t *tokens = nullptr;  // [B, 4 * topk] kept token indices (token-budget output), or NULL
+  int T = 1;                  // query tokens per request: tokens are listed up to p0 = L - T
   int32_t *scores;   // [B, max_blocks]
 };
 
@@ -137,10 +139,28 @@ __device__ __forceinline__ void append_cand(bool take, unsigned long long x, Sel
   }
 }
 
+// Output row entries of the kept block `blk` at rank `pos` (< K) in
+// ascending order: out[pos] = blk and, for the token-budget output, the
+// four token slots 4*pos .. 4*pos+3 hold 4*blk + j where that token is at
+// most p0 (request-relative position of query token 0), else -1.  Only the
+// block holding p0 can be cut, and it is the last kept block, so the -1 of
+// a row all sit at its end.
+__device__ __forceinline__ void put_block(int32_t *out, int32_t *tok, int pos, int blk, int p0) {
+  if (out) out[pos] = blk;
+  if (tok) {
+    int4 v;
+    v.x = 4 * blk <= p0 ? 4 * blk : -1;
+    v.y = 4 * blk + 1 <= p0 ? 4 * blk + 1 : -1;
+    v.z = 4 * blk + 2 <= p0 ? 4 * blk + 2 : -1;
+    v.w = 4 * blk + 3 <= p0 ? 4 * blk + 3 : -1;
+    *reinterpret_cast<int4 *>(tok + 4 * pos) = v;
+  }
+}
+
 // Writes the set bits of bits[0 .. ceil(n/32)) as ascending indices:
 // exactly K bits are set.
-__device__ void write_from_bits(const uint32_t *bits, int n, int K, int32_t *out, SelSmem &sm,
-                                int tid) {
+__device__ void write_from_bits(const uint32_t *bits, int n, int K, int32_t *out, int32_t *tok,
+                                int p0, SelSmem &sm, int tid) {
   const int W = (n + 31) >> 5;
   const int per = (W + kSelThreads - 1) / kSelThreads;
   const int w0 = min(W, tid * per), w1 = min(W, w0 + per);
@@ -152,7 +172,7 @@ __device__ void write_from_bits(const uint32_t *bits, int n, int K, int32_t *out
     while (m) {
       const int b = __ffs(m) - 1;
       m &= m - 1u;
-      if (pos < K) out[pos] = w * 32 + b;
+      if (pos < K) put_block(out, tok, pos, w * 32 + b, p0);
       ++pos;
     }
   }
@@ -384,13 +404,14 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
 
 // Writes the K distinct kept indices in ascending order: by rank counting
 // for small K, by a bitonic sort otherwise.
-__device__ void write_ascending(int *keep, int K, int32_t *out, SelSmem &sm, int tid) {
+__device__ void write_ascending(int *keep, int K, int32_t *out, int32_t *tok, int p0, SelSmem &sm,
+                                int tid) {
   if (K <= 1024) {
     for (int i = tid; i < K; i += kSelThreads) {
       const int x = keep[i];
       int rank = 0;
       for (int j = 0; j < K; ++j) rank += (keep[j] < x);
-      out[rank] = x;
+      put_block(out, tok, rank, x, p0);
     }
     return;
   }
@@ -398,7 +419,7 @@ __device__ void write_ascending(int *keep, int K, int32_t *out, SelSmem &sm, int
   for (int i = K + tid; i < kp2; i += kSelThreads) keep[i] = 0x7fffffff;
   __syncthreads();
   bitonic_sort_i32(keep, kp2, tid);
-  for (int i = tid; i < K; i += kSelThreads) out[i] = keep[i];
+  for (int i = tid; i < K; i += kSelThreads) put_block(out, tok, i, keep[i], p0);
 }
 
 // The two passes of the selection over a score row: a histogram of the
@@ -447,10 +468,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
   const int tid = threadIdx.x;
   const int n = request_blocks(p, r, tid == 0);
   const int K = p.topk;
-  int32_t *out = p.sel + (long long)r * K;
+  int32_t *tok = p.tokens ? p.tokens + (long long)r * 4 * K : nullptr;
+  const int p0 = p.ctx_lens[r] - p.T;
+  int32_t *out = p.sel ? p.sel + (long long)r * K : nullptr;
   const int32_t *sc = p.scores + (long long)r * p.max_blocks;
   if (n <= K) {
-    for (int i = tid; i < K; i += kSelThreads) out[i] = i < n ? i : -1;
+    for (int i = tid; i < K; i += kSelThreads) {
+      if (i < n) {
+        put_block(out, tok, i, i, p0);
+      } else {
+        if (out) out[i] = -1;
+        if (tok) *reinterpret_cast<int4 *>(tok + 4 * i) = make_int4(-1, -1, -1, -1);
+      }
+    }
     return;
   }
   // kept blocks go to a bitmap when the request fits it, else to a list
@@ -492,8 +522,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
       __syncthreads();
     }
   }
-  if (use_bits) write_from_bits(sm.bits, n, K, out, sm, tid);
-  else write_ascending(keep, K, out, sm, tid);
+  if (use_bits) write_from_bits(sm.bits, n, K, out, tok, p0, sm, tid);
+  else write_ascending(keep, K, out, tok, p0, sm, tid);
 }
 
 // ------------------------------------------------------------- the scan --

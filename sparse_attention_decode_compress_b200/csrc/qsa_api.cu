@@ -300,22 +300,30 @@ size_t qsa_index_topk_workspace_bytes(int32_t B, int32_t max_blocks) {
   return kTicketBytes + align_up((size_t)B * (size_t)max_blocks * sizeof(int32_t));
 }
 
-qsa_status qsa_index_topk(const qsa_cache *cache, int32_t B, const int8_t *q_idx,
-                          const int32_t *ctx_lens, const int32_t *n_sel, int32_t max_blocks,
-                          int32_t topk, int32_t *sel, int32_t *scores, void *workspace,
-                          size_t workspace_bytes, qsa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of qsa_index_topk and qsa_index_topk_tokens: validation, then
+// scan + selection.  sel and/or tokens receive the output rows.
+qsa_status index_topk_call(const qsa_cache *cache, int32_t B, const int8_t *q_idx,
+                           const int32_t *ctx_lens, const int32_t *n_sel, int32_t T,
+                           int32_t max_blocks, int32_t topk, int32_t *sel, int32_t *tokens,
+                           int32_t *scores, void *workspace, size_t workspace_bytes,
+                           qsa_stream_t stream) {
   qsa_status st = check_cache(cache);
   if (st != QSA_OK) return st;
   if (B < 0) return QSA_ERR_INVALID_ARG;
   if (topk < 1 || topk > qsa::topk::kMaxTopk) return QSA_ERR_INVALID_ARG;
   if (max_blocks < 1 || max_blocks > (1 << 24)) return QSA_ERR_INVALID_ARG;
+  if (T < 1 || T > qsa::dec::kMaxT) return QSA_ERR_INVALID_ARG;
   if (B == 0) return QSA_OK;
   if (B > 0x7fffffff / 2) return QSA_ERR_UNSUPPORTED;
-  if (!q_idx || !ctx_lens || !sel || !workspace || !cache->kc) return QSA_ERR_INVALID_ARG;
+  if (!q_idx || !ctx_lens || !(sel || tokens) || !workspace || !cache->kc) return QSA_ERR_INVALID_ARG;
   if (cache->idx_dim != 32 && cache->idx_dim != 64 && cache->idx_dim != 128)
     return QSA_ERR_UNSUPPORTED;
   if (!aligned(cache->kc, 16) || !aligned(q_idx, 4) || !aligned(workspace, 16) ||
-      (scores && !aligned(scores, 4)))
+      (scores && !aligned(scores, 4)) || (tokens && !aligned(tokens, 16)))
     return QSA_ERR_INVALID_ARG;
   const size_t need = scores ? kTicketBytes : qsa_index_topk_workspace_bytes(B, max_blocks);
   if (workspace_bytes < need) return QSA_ERR_INVALID_ARG;
@@ -329,6 +337,8 @@ qsa_status qsa_index_topk(const qsa_cache *cache, int32_t B, const int8_t *q_idx
   p.max_blocks = max_blocks;
   p.topk = topk;
   p.sel = sel;
+  p.tokens = tokens;
+  p.T = T;
   p.scores = scores ? scores
                     : reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + kTicketBytes);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -341,6 +351,29 @@ qsa_status qsa_index_topk(const qsa_cache *cache, int32_t B, const int8_t *q_idx
     default: return P == 64 ? launch_index_topk<128, 16>(p, s)
                   : P == 16 ? launch_index_topk<128, 4>(p, s) : launch_index_topk<128, 0>(p, s);
   }
+}
+
+}  // namespace
+
+extern "C" {
+
+qsa_status qsa_index_topk(const qsa_cache *cache, int32_t B, const int8_t *q_idx,
+                          const int32_t *ctx_lens, const int32_t *n_sel, int32_t max_blocks,
+                          int32_t topk, int32_t *sel, int32_t *scores, void *workspace,
+                          size_t workspace_bytes, qsa_stream_t stream) {
+  return index_topk_call(cache, B, q_idx, ctx_lens, n_sel, 1, max_blocks, topk, sel, nullptr,
+                         scores, workspace, workspace_bytes, stream);
+}
+
+qsa_status qsa_index_topk_tokens(const qsa_cache *cache, int32_t B, const int8_t *q_idx,
+                                 const int32_t *ctx_lens, const int32_t *n_sel, int32_t T,
+                                 int32_t max_blocks, int32_t budget, int32_t *tokens,
+                                 int32_t *sel, int32_t *scores, void *workspace,
+                                 size_t workspace_bytes, qsa_stream_t stream) {
+  if (budget < 4 || budget % 4 != 0) return QSA_ERR_INVALID_ARG;
+  if (B > 0 && !tokens) return QSA_ERR_INVALID_ARG;
+  return index_topk_call(cache, B, q_idx, ctx_lens, n_sel, T, max_blocks, budget / 4, sel, tokens,
+                         scores, workspace, workspace_bytes, stream);
 }
 
 size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32_t Hkv,

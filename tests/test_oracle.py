@@ -83,6 +83,41 @@ def test_hand_mtp(hand):
     assert ref.token_set(sel, L, T, 1).tolist() == hand["mtp_tokens_t1"]
 
 
+def test_hand_token_budget(hand):
+    k = np.array(hand["k_idx"], dtype=np.int8)
+    L = k.shape[0]
+    s = ref.block_scores(np.array(hand["q_idx"], dtype=np.int8), ref.compress_keys(k))
+    assert ref.selection_tokens(ref.select_blocks(s, 2), L, 1, 8).tolist() == hand["budget8_tokens_T1"]
+    assert ref.selection_tokens(ref.select_blocks(s, 4), L, 1, 16).tolist() == hand["budget16_tokens_T1"]
+    T = hand["mtp_T"]
+    s_mtp = ref.block_scores(np.array(hand["q_idx"], dtype=np.int8), ref.compress_keys(k),
+                             ref.selection_width(L, T))
+    assert ref.selection_tokens(ref.select_blocks(s_mtp, 1), L, T, 4).tolist() == hand["budget4_tokens_mtp"]
+
+
+def test_token_budget_properties_brute_force():
+    """Every listed token lies in a selected block and at or before p0; the
+    row is ascending with its -1 at the end; nothing visible is left out;
+    the listed tokens are query token 0's attended set."""
+    rng = np.random.default_rng(5)
+    for _ in range(300):
+        L = int(rng.integers(1, 60))
+        T = int(rng.integers(1, 5))
+        n = (L + 3) // 4
+        topk = int(rng.integers(1, 12))
+        sel = ref.select_blocks(rng.integers(-5, 5, n), topk)
+        budget = 4 * topk
+        row = ref.selection_tokens(sel, L, T, budget)
+        p0 = L - T
+        kept = [int(b) for b in sel if b >= 0]
+        listed = [int(t) for t in row if t >= 0]
+        expect = [4 * b + j for b in kept for j in range(4) if 4 * b + j <= p0]
+        assert listed == sorted(expect)
+        assert all(t == -1 for t in row[len(listed):])
+        assert all(t // 4 in kept and t <= p0 for t in listed)
+        assert listed == ref.token_set(sel, L, T, 0).tolist()
+
+
 # --------------------------------------------------------------------------
 # Value decoding vs the library conversions
 # --------------------------------------------------------------------------
