@@ -284,6 +284,65 @@ qsa_status qsa_index_topk_noalloc(const qsa_cache *cache, int32_t B, const int8_
  */
 qsa_status qsa_get_device_error(qsa_stream_t stream, uint32_t *flags_out);
 
+/*
+ * Decode session — one decode step per call, host buffers in and out, with
+ * the transfers overlapped with the kernels.
+ *
+ * The pages' path runs inside a serving runtime that owns the transfers;
+ * they have no counterpart for this call.  It exists so that an end-to-end
+ * step (inputs from host memory, o / lse back to host memory) costs no more
+ * than the kernels:
+ * - The session owns two slots of device input and output buffers, plus
+ *   the selection, split partials and workspaces.
+ * - Its upload stream copies step k+1's inputs while step k computes on the
+ *   compute stream, and its download stream copies step k-1's o / lse back.
+ *   Events order the three streams.
+ * - A step runs exactly qsa_compress_append, qsa_index_topk,
+ *   qsa_sparse_decode (sm_scale, num_splits) and qsa_lse_merge.
+ *
+ * qsa_session_create allocates every buffer (cudaMalloc, the decode
+ * workspace zero-filled) and two non-blocking streams. It copies *cache
+ * (the caches stay the caller's).
+ *   T, Hq, topk, num_splits, max_blocks as for the calls above
+ *   q_dtype         QSA_BF16 (bf16 / fp8 caches) or QSA_F32 (fp32 caches)
+ *   max_new_tokens  bound on cu_new[B] (tokens appended per step)
+ *   compute_stream  stream for the kernels, or NULL for a session-owned one
+ *   *out            receives the session
+ *
+ * qsa_session_step_host enqueues one step and returns without waiting:
+ *   pos0 [B], cu_new [B+1], k_new [cu_new[B], d], q_idx [B, d],
+ *   q [B, T, Hq, D] of q_dtype, ctx_lens [B], n_sel [B] or NULL
+ *     host inputs; cu_new is also read on the host
+ *   o [B, T, Hq, D] float32, lse [B, T, Hq] float32
+ *     host outputs
+ * Host buffers should be pinned (cudaHostAlloc or registered) for the
+ * copies to overlap. Pageable memory works, but the copies then block.
+ * Inputs must stay unchanged and outputs untouched until
+ * qsa_session_synchronize returns.
+ *
+ * qsa_session_streams reports the three streams, for events and waits.
+ * qsa_session_synchronize waits for every enqueued step.
+ * qsa_session_destroy synchronises and frees the session.
+ *
+ * Errors: QSA_ERR_INVALID_ARG for bad sizes, null pointers or cu_new[B] >
+ * max_new_tokens; QSA_ERR_CUDA when an allocation, copy or stream call
+ * fails; otherwise the status of the failing library call.
+ */
+typedef struct qsa_session qsa_session;
+
+qsa_status qsa_session_create(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
+                              int32_t q_dtype, int32_t topk, int32_t num_splits,
+                              int32_t max_blocks, int32_t max_new_tokens, float sm_scale,
+                              qsa_stream_t compute_stream, qsa_session **out);
+qsa_status qsa_session_step_host(qsa_session *s, const int32_t *pos0, const int32_t *cu_new,
+                                 const int8_t *k_new, const int8_t *q_idx, const void *q,
+                                 const int32_t *ctx_lens, const int32_t *n_sel, float *o,
+                                 float *lse);
+qsa_status qsa_session_streams(const qsa_session *s, qsa_stream_t *h2d, qsa_stream_t *compute,
+                               qsa_stream_t *d2h);
+qsa_status qsa_session_synchronize(qsa_session *s);
+qsa_status qsa_session_destroy(qsa_session *s);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,13 +1,14 @@
 """Decode-time Qwen Sparse Attention (QSA) on B200: a C-ABI library of
 hand-written sm_100a kernels (libqsa.so) and its thin PyTorch binding."""
-from .api import (QSACache, QSAError, new_workspace, qsa_compress_append, qsa_get_device_error,
-                  qsa_index_topk, qsa_index_topk_noalloc, qsa_index_topk_workspace_bytes,
-                  qsa_lse_merge, qsa_sparse_decode, qsa_sparse_decode_workspace_bytes)
+from .api import (QSACache, QSAError, QSASession, new_workspace, qsa_compress_append,
+                  qsa_get_device_error, qsa_index_topk, qsa_index_topk_noalloc,
+                  qsa_index_topk_tokens, qsa_index_topk_workspace_bytes, qsa_lse_merge,
+                  qsa_sparse_decode, qsa_sparse_decode_workspace_bytes)
 from .decode import QSADecodeStep
 
 __all__ = [
-    "QSACache", "QSAError", "QSADecodeStep", "new_workspace", "qsa_compress_append",
-    "qsa_get_device_error", "qsa_index_topk", "qsa_index_topk_noalloc",
+    "QSACache", "QSAError", "QSADecodeStep", "QSASession", "new_workspace", "qsa_compress_append",
+    "qsa_get_device_error", "qsa_index_topk", "qsa_index_topk_noalloc", "qsa_index_topk_tokens",
     "qsa_index_topk_workspace_bytes", "qsa_lse_merge",
     "qsa_sparse_decode", "qsa_sparse_decode_workspace_bytes",
 ]

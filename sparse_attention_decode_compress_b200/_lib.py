@@ -47,6 +47,14 @@ SIGNATURES = {
                                         c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
                                         c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "qsa_get_device_error": (c_int32, [c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
+    "qsa_session_create": (c_int32, [ctypes.POINTER(QsaCacheStruct), c_int32, c_int32, c_int32,
+                                     c_int32, c_int32, c_int32, c_int32, c_int32, c_float,
+                                     c_void_p, ctypes.POINTER(c_void_p)]),
+    "qsa_session_step_host": (c_int32, [c_void_p] * 10),
+    "qsa_session_streams": (c_int32, [c_void_p, ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p),
+                                      ctypes.POINTER(c_void_p)]),
+    "qsa_session_synchronize": (c_int32, [c_void_p]),
+    "qsa_session_destroy": (c_int32, [c_void_p]),
 }
 
 _lib = None

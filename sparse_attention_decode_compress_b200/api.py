@@ -236,6 +236,72 @@ def qsa_lse_merge(o_part: torch.Tensor, lse_part: torch.Tensor, o: torch.Tensor,
                              _stream(stream)), "qsa_lse_merge")
 
 
+class QSASession:
+    """Decode steps from host buffers to host buffers (qsa_session_*): the
+    library owns the device buffers and overlaps each step's uploads and
+    downloads with the kernels of its neighbours.  Host tensors should be
+    pinned; they must stay unchanged (inputs) and untouched (outputs) until
+    synchronize() returns."""
+
+    def __init__(self, cache: QSACache, B: int, T: int, Hq: int, topk: int, num_splits: int,
+                 max_blocks: int, max_new_tokens: int, sm_scale: float,
+                 q_dtype=torch.bfloat16, stream=None):
+        self.cache = cache  # keeps the caches alive
+        self._struct = cache.struct()
+        self.B, self.T, self.Hq, self.topk = B, T, Hq, topk
+        self.D = cache.k_cache.shape[-1]
+        self.d = cache.kc.shape[-1]
+        self.q_dtype = q_dtype
+        qd = {torch.float32: _lib.QSA_F32, torch.bfloat16: _lib.QSA_BF16}[q_dtype]
+        lib = _lib.load()
+        h = ctypes.c_void_p()
+        cs = stream.cuda_stream if stream is not None else None
+        _check(lib.qsa_session_create(ctypes.byref(self._struct), B, T, Hq, qd, topk, num_splits,
+                                      max_blocks, max_new_tokens, float(sm_scale), cs,
+                                      ctypes.byref(h)), "qsa_session_create")
+        self._h = h
+
+    def step(self, pos0, cu_new, k_new, q_idx, q, ctx_lens, n_sel, o, lse) -> None:
+        B, T, Hq, D, d = self.B, self.T, self.Hq, self.D, self.d
+        want = [(pos0, torch.int32, (B,)), (cu_new, torch.int32, (B + 1,)),
+                (q_idx, torch.int8, (B, d)), (q, self.q_dtype, (B, T, Hq, D)),
+                (ctx_lens, torch.int32, (B,)), (o, torch.float32, (B, T, Hq, D)),
+                (lse, torch.float32, (B, T, Hq))]
+        if n_sel is not None:
+            want.append((n_sel, torch.int32, (B,)))
+        for t, dt, shape in want:
+            if t.is_cuda or t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"host tensor of dtype {dt} and shape {shape} expected")
+        if (k_new.is_cuda or k_new.dtype != torch.int8 or k_new.dim() != 2 or
+                k_new.shape[1] != d or not k_new.is_contiguous()):
+            raise ValueError("k_new must be a contiguous host int8 tensor [N, d]")
+        p = lambda t: None if t is None else t.data_ptr()
+        _check(_lib.load().qsa_session_step_host(self._h, p(pos0), p(cu_new), p(k_new), p(q_idx),
+                                                 p(q), p(ctx_lens), p(n_sel), p(o), p(lse)),
+               "qsa_session_step_host")
+
+    def streams(self) -> tuple[int, int, int]:
+        """(upload, compute, download) stream handles."""
+        a, b, c = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+        _check(_lib.load().qsa_session_streams(self._h, ctypes.byref(a), ctypes.byref(b),
+                                               ctypes.byref(c)), "qsa_session_streams")
+        return a.value or 0, b.value or 0, c.value or 0
+
+    def synchronize(self) -> None:
+        _check(_lib.load().qsa_session_synchronize(self._h), "qsa_session_synchronize")
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _lib.load().qsa_session_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
 def qsa_get_device_error(stream=None) -> tuple[int, int]:
     """Synchronises the stream; returns (status, flag bits) and clears the
     device error word."""

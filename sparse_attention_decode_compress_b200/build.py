@@ -32,13 +32,15 @@ def needs_rebuild() -> bool:
 
 
 def build_library(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    """Compiles csrc/qsa_api.cu (which includes every kernel) into libqsa.so."""
+    """Compiles csrc/qsa_api.cu (which includes every kernel) and
+    csrc/qsa_session.cu (the host-side decode session) into libqsa.so."""
     if not force and not needs_rebuild():
         return LIB_PATH
     os.makedirs(LIB_DIR, exist_ok=True)
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB_PATH + ".tmp"
-    cmd = [nvcc, *NVCC_FLAGS, "-I" + INCLUDE, "-o", tmp, os.path.join(CSRC, "qsa_api.cu")]
+    cmd = [nvcc, *NVCC_FLAGS, "-I" + INCLUDE, "-o", tmp, os.path.join(CSRC, "qsa_api.cu"),
+           os.path.join(CSRC, "qsa_session.cu")]
     if ptxas_info:
         cmd.insert(1, "-Xptxas=-v")
     if verbose:
