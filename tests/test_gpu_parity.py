@@ -123,6 +123,34 @@ def test_extreme_scores_order_exactly():
     _check_all(b, step, cache, 2)
 
 
+SHAPES = [
+    # (workload, overrides, context lengths, splits)
+    ("b32_32k", dict(topk=64), [9000, 3001], 2),
+    ("b32_32k", dict(topk=2048), [12345, 9001], 2),
+    ("b32_32k", dict(topk=4096), [20000, 17000], 3),
+    ("b32_32k", dict(D=64), [9000, 5003], 2),
+    ("b32_32k", dict(Hq=32, Hkv=4), [9000, 7777], 2),
+    ("b32_32k", dict(Hq=8, Hkv=8), [9000, 4097], 2),
+    ("b32_32k", dict(Hq=32, Hkv=2), [9000, 6001], 2),
+    ("b32_32k", dict(T=2), [9000, 6002], 2),
+    ("b32_32k", dict(T=3), [9000, 6003], 2),
+    ("b32_32k", dict(page_size=32), [9000, 6007], 2),
+    ("b32_32k", dict(d_idx=64), [9000, 6009], 2),
+    ("b32_32k", dict(page_size=16, d_idx=32), [9000, 6011], 16),
+    ("mixed_fp8", dict(D=64), [9000, 5005], 4),
+]
+
+
+@pytest.mark.parametrize("name,over,lens,S", SHAPES)
+def test_other_shapes(name, over, lens, S):
+    """Head counts, head and indexer dims, page sizes, query tokens, top-k
+    widths and split counts beyond the named workloads."""
+    w = replace(WORKLOADS[name], **over)
+    b = make_batch(w, "cuda", ctx_lens=lens, seed=17)
+    step, cache = H.run_gpu(b, S)
+    _check_all(b, step, cache, S)
+
+
 def test_split_count_invariance():
     w = WORKLOADS["b128_256k"]
     b = make_batch(w, "cuda", ctx_lens=[40000, 30001], seed=21)
