@@ -106,6 +106,18 @@ def algorithmic_bytes(w, L: int, num_splits: int) -> dict:
                 total=idx + dec + merge + append)
 
 
+def workload_config(w, num_splits: int, world: int) -> dict:
+    """The `config` object of the JSON line (both arms)."""
+    kind, *a = w.ctx.split(":")
+    return {"workload": w.name, "description": w.description, "global_batch": w.batch * world,
+            "seq_len": int(a[-1]), "query_tokens": w.T, "kv_splits": num_splits,
+            "topk_blocks": w.topk, "page_size": w.page_size,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (2 GiB compressed keys read per step)",
+            "timing": "value: K back-to-back steps; kernel_ms and roofline: a second "
+                      "K-step pass with events between the kernels"}
+
+
 def index_topk_traffic(batch: int):
     """DRAM bytes of one qsa_index_topk launch from the committed ncu capture
     (profiles/roofline_traffic.json), scaled by requests; None when the
@@ -463,13 +475,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "warmup": args.warmup, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.kv_dtype if w.kv_dtype != "f32" else "f32",
         "data": "synthetic (seeded; stands in for the pages' 256k-context serving trace)",
-        "config": {"workload": args.workload, "description": w.description, "global_batch": B * world,
-                   "seq_len": int(L_host.max()), "query_tokens": T, "kv_splits": S,
-                   "topk_blocks": w.topk, "page_size": w.page_size,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (2 GiB compressed keys read per step)",
-                   "timing": "value: K back-to-back steps; kernel_ms and roofline: a second "
-                             "K-step pass with events between the kernels"},
+        "config": workload_config(w, S, world),
         "hbm_gbs": round(hbm, 1),
         "hbm_pct_of_peak": round(100 * hbm / peaks["hbm_gbs"], 2),
         "hbm_pct_of_nominal_8tbs": round(100 * hbm / 8000.0, 2),
@@ -503,7 +509,8 @@ def main(argv=None):
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(1e3 * res["seconds"] / args.steps, 3), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
-                "data": "synthetic", "config": {"workload": args.workload, "kv_splits": args.splits},
+                "data": "synthetic (seeded; stands in for the pages' 256k-context serving trace)",
+                "config": workload_config(w, args.splits, max(1, args.gpus)),
                 "cpu_baseline": {"value": round(res["value"], 4), "unit": UNIT, "cores": res["cores"],
                                  "kind": "oracle",
                                  "sample": f"{res['queries']} decode steps of {args.workload} (one "
