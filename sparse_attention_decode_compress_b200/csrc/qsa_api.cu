@@ -15,6 +15,7 @@
 #include "index_topk.cuh"
 #include "sparse_decode.cuh"
 #include "sparse_decode_warp.cuh"
+#include "sparse_decode_group.cuh"
 #include "lse_merge.cuh"
 
 namespace {
@@ -232,13 +233,41 @@ qsa_status launch_decode_f32(qsa::dec::Params p, cudaStream_t stream) {
   return launch(true, kernel, grid, dim3(qsa::dec::kThreads), smem, stream, p);
 }
 
+// More than 8 query rows: groups of GW = NT warps, one per 8-row tile,
+// sharing a ring of NS = 2 * GW stages (12 warps per SM).
+template <int D, bool FP8, int GW>
+qsa_status launch_decode_group(qsa::dec::Params p, cudaStream_t stream) {
+  constexpr int NW = 12;
+  constexpr int NS = 2 * GW;
+  static bool done[kMaxDevices] = {false};
+  static int blocks_per_sm[kMaxDevices] = {0};
+  auto kernel = qsa::dec::sparse_decode_group_kernel<D, FP8, NW, NS, GW>;
+  const size_t smem = sizeof(qsa::dec::GroupSmem<D, FP8, NW, NS, GW>) + 128;
+  const int dev = current_device();
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (prepare_kernel(kernel, smem, done) != cudaSuccess) return QSA_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices && !blocks_per_sm[dev]) {
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, NW * 32, smem) != cudaSuccess)
+        return QSA_ERR_CUDA;
+      blocks_per_sm[dev] = n > 0 ? n : 1;
+    }
+  }
+  const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
+  const int ctas = bps * sm_count(dev);
+  p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, (long long)ctas * (NW / GW));
+  p.nch = decode_chunk_slots(p.topk, p.S, p.chunk);
+  return launch(true, kernel, dim3(ctas), dim3(NW * 32), smem, stream, p);
+}
+
 template <int D, bool FP8>
 qsa_status dispatch_decode_nt(const qsa::dec::Params &p, int NT, cudaStream_t stream) {
   switch (NT) {
     case 1: return launch_decode_warp<D, 1, FP8>(p, stream);
-    case 2: return launch_decode_warp<D, 2, FP8>(p, stream);
-    case 3: return launch_decode_warp<D, 3, FP8>(p, stream);
-    default: return launch_decode_warp<D, 4, FP8>(p, stream);
+    case 2: return launch_decode_group<D, FP8, 2>(p, stream);
+    case 3: return launch_decode_group<D, FP8, 3>(p, stream);
+    default: return launch_decode_group<D, FP8, 4>(p, stream);
   }
 }
 
