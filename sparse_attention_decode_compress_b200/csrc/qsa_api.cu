@@ -162,18 +162,22 @@ int decode_chunk_slots(int topk, int S, int chunk) {
 }
 
 // Chunk size of the persistent decode: the largest work items that still
-// give every worker warp at most one of them (one wave, no tail of second
-// items), within [kMinChunkBlocks, kChunkBlocks].  A batch with more
-// (request, kv head) pairs than warps takes the largest chunks.  (Two or
-// three smaller chunks per warp, balanced through the work counter,
-// measured ~30% slower: each chunk's fixed plan / metadata / epilogue
-// latency is paid again.)
-int decode_chunk_blocks(int B, int Hkv, int topk, int S, long long workers) {
+// give every worker at most one of them (one wave, no tail of second
+// items), within [kMinChunkBlocks, cap].  A (request, kv head) pair gets
+// floor(workers / pairs) workers, c = that / S per split; its splits hold
+// about (topk + 2) / S entries each, with 20% added for splits that hold
+// more than their share, so that each split takes c chunks.  A batch with
+// more pairs than workers takes the largest chunks.  (Two or three smaller
+// chunks per warp, balanced through the work counter, measured ~30% slower:
+// each chunk's fixed plan / metadata / epilogue latency is paid again.)
+int decode_chunk_blocks(int B, int Hkv, int topk, int S, long long workers, int cap) {
   const long long pairs = (long long)B * Hkv;
-  const long long per_pair = workers / (pairs > 0 ? pairs : 1);
-  const long long n_chunks = per_pair - (S - 1);
-  int chunk = qsa::dec::kChunkBlocks;
-  if (n_chunks > 0) chunk = (int)std::min<long long>(chunk, (topk + 2 + n_chunks - 1) / n_chunks);
+  const long long per_split = workers / (pairs > 0 ? pairs : 1) / S;
+  int chunk = cap;
+  if (per_split > 0) {
+    const long long share = ((long long)topk + 2) * 6 / (5 * S);  // split share with 20% headroom
+    chunk = (int)std::min<long long>(chunk, (share + per_split - 1) / per_split);
+  }
   return std::max(chunk, qsa::dec::kMinChunkBlocks);
 }
 
@@ -213,7 +217,8 @@ qsa_status launch_decode_warp(qsa::dec::Params p, cudaStream_t stream) {
   }
   const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
   const int ctas = bps * sm_count(dev);
-  p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, (long long)ctas * NW);
+  p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, (long long)ctas * NW,
+                                qsa::dec::kChunkBlocks);
   p.nch = decode_chunk_slots(p.topk, p.S, p.chunk);
   return launch(true, kernel, dim3(ctas), dim3(NW * 32), smem, stream, p);
 }
@@ -256,7 +261,8 @@ qsa_status launch_decode_group(qsa::dec::Params p, cudaStream_t stream) {
   }
   const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
   const int ctas = bps * sm_count(dev);
-  p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, (long long)ctas * (NW / GW));
+  p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, (long long)ctas * (NW / GW),
+                                qsa::dec::kGroupChunkBlocks);
   p.nch = decode_chunk_slots(p.topk, p.S, p.chunk);
   return launch(true, kernel, dim3(ctas), dim3(NW * 32), smem, stream, p);
 }

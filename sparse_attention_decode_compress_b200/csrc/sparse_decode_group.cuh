@@ -21,9 +21,13 @@
 namespace qsa {
 namespace dec {
 
+// Chunk capacity of a group: a group streams GW times faster than a warp
+// of the same rows, so it takes whole splits when the batch is small.
+constexpr int kGroupChunkBlocks = 512;
+
 template <int D, bool FP8, int NW, int NS, int GW>
 struct GroupSmem {
-  WarpState<D, FP8, NS> g[NW / GW];
+  WarpState<D, FP8, NS, kGroupChunkBlocks> g[NW / GW];
   int item[NW / GW];
   int last[NW / GW];
 };
@@ -37,7 +41,7 @@ __device__ void fill_meta_group(const Params &p, const Plan &pl, int r, int g, W
   const int P = p.c.page_size, Hkv = p.c.num_kv_heads;
   const bool pow2 = (P & (P - 1)) == 0;
   const int lgP = 31 - __clz(P);
-  for (int kb = tig; kb < kChunkBlocks; kb += nthr) {
+  for (int kb = tig; kb < WS::kCap; kb += nthr) {
     const int e = pl.e_begin + kb;
     const int b = (e < pl.e_end) ? ext_block(sel_r, pl, e) : -1;
     int pg = -1;
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
   constexpr int NG = NW / GW;
   extern __shared__ uint8_t smem_raw[];
   using SM = GroupSmem<D, FP8, NW, NS, GW>;
-  using WS = WarpState<D, FP8, NS>;
+  using WS = WarpState<D, FP8, NS, kGroupChunkBlocks>;
   SM &sm = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = warp / GW, wig = warp % GW;  // group, and this warp's 8-row tile

@@ -24,17 +24,18 @@ constexpr int kCounterInts = 64;  // workspace header: [0] next item, [1] finish
 
 // Shared-memory layout of one worker warp: a ring of NS 16-token K/V stages,
 // an fp8 -> bf16 conversion stage and the chunk's token metadata.
-template <int D, bool FP8, int NS>
+template <int D, bool FP8, int NS, int CAP = kChunkBlocks>
 struct WarpState {
   static constexpr int kRowBytes = D * (FP8 ? 1 : 2);
+  static constexpr int kCap = CAP;  // micro-blocks a chunk may hold
   alignas(128) uint8_t ring[NS][2][kTokW * kRowBytes];
   alignas(128) uint8_t cvt[FP8 ? 2 : 1][FP8 ? kTokW * D * 2 : 16];
-  int boff[kChunkBlocks];  // cache row (token, head g) of each micro-block's first token
+  int boff[CAP];  // cache row (token, head g) of each micro-block's first token
   // byte j of word b: visibility bits of token j of micro-block b (bit t:
   // visible to query token t); a token visible to none is not loaded
-  uint32_t vmask4[kChunkBlocks];
-  float ks[FP8 ? kChunkBlocks : 1];  // fp8 scales of each micro-block's page
-  float vs[FP8 ? kChunkBlocks : 1];
+  uint32_t vmask4[CAP];
+  float ks[FP8 ? CAP : 1];  // fp8 scales of each micro-block's page
+  float vs[FP8 ? CAP : 1];
   Plan pl;
   __device__ __forceinline__ unsigned vmask(int tok) const {
     return reinterpret_cast<const unsigned char *>(vmask4)[tok];
