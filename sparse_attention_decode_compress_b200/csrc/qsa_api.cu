@@ -235,7 +235,7 @@ qsa_status launch_decode_warp(qsa::dec::Params p, cudaStream_t stream) {
 template <int D>
 qsa_status launch_decode_f32(qsa::dec::Params p, cudaStream_t stream) {
   static bool done[kMaxDevices] = {false};
-  p.chunk = qsa::dec::kChunkBlocks;  // one CTA per chunk slot
+  p.chunk = qsa::dec::kMinChunkBlocks;  // one CTA per chunk slot: many small ones
   p.nch = decode_chunk_slots(p.topk, p.S, p.chunk);
   const dim3 grid((unsigned)p.nch, (unsigned)p.c.num_kv_heads, (unsigned)p.B);
   auto kernel = qsa::dec::sparse_decode_f32_kernel<D>;

@@ -373,7 +373,7 @@ struct F32Smem {
   Plan pl;
   float o[kMaxRows * D];
   float lse[kMaxRows];
-  float scratch[kMaxRows * (4096 / kChunkBlocks + 2 + kMaxSplits)];  // chunk = kChunkBlocks
+  float scratch[kMaxRows * (4096 / kMinChunkBlocks + 2 + kMaxSplits)];  // nch * M floats
   int flag;
 };
 
