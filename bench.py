@@ -42,6 +42,8 @@ def parse_args(argv=None):
                     help="override the workload's batch (profiling runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the steps as eager launches instead of one CUDA graph replay")
     ap.add_argument("--cpu-queries", type=int, default=300,
                     help="oracle queries timed for the CPU baseline")
     return ap.parse_args(argv)
@@ -114,8 +116,9 @@ def workload_config(w, num_splits: int, world: int) -> dict:
             "topk_blocks": w.topk, "page_size": w.page_size,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": "inputs larger than L2 (2 GiB compressed keys read per step)",
-            "timing": "value: K back-to-back steps; kernel_ms and roofline: a second "
-                      "K-step pass with events between the kernels"}
+            "timing": "value: K back-to-back steps (one CUDA graph of the K steps, replayed "
+                      "once after an untimed replay; --no-graph: eager launches); kernel_ms and "
+                      "roofline: a second, eager K-step pass with events between the kernels"}
 
 
 def index_topk_traffic(batch: int):
@@ -376,7 +379,19 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         sampler.start()
         time.sleep(0.3)
     K = args.steps
-    # timed region 1: K whole steps back to back (the value)
+    # timed region 1: K whole steps back to back (the value), as one CUDA
+    # graph holding the K steps (replayed once untimed first), or as eager
+    # launches with --no-graph
+    graph = None
+    if not args.no_graph:
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            for k in range(K):
+                one_step()
+        graph.replay()
+        torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -384,14 +399,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     sampler.mark("t0")
     t_start.record(stream)
-    for k in range(K):
-        one_step()
+    if graph is not None:
+        graph.replay()
+    else:
+        for k in range(K):
+            one_step()
     t_end.record(stream)
     torch.cuda.synchronize()
     sampler.mark("t1")
     if world > 1:
         dist.barrier()
     ms = t_start.elapsed_time(t_end)
+    del graph
     # timed region 2: the same K steps with events between the kernels, for
     # the per-launch durations of the roofline (an event between two kernels
     # costs the step a few microseconds, so the value comes from region 1)
