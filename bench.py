@@ -42,6 +42,10 @@ def parse_args(argv=None):
                     help="override the workload's batch (profiling runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--dcp", action="store_true",
+                    help="decode context parallelism: the ranks share one batch, rank k attends "
+                         "split k of N and the partials are all-gathered (strong scaling); "
+                         "default: independent replicas (weak scaling)")
     ap.add_argument("--no-graph", action="store_true",
                     help="time the steps as eager launches instead of one CUDA graph replay")
     ap.add_argument("--cpu-queries", type=int, default=300,
@@ -108,13 +112,17 @@ def algorithmic_bytes(w, L: int, num_splits: int) -> dict:
                 total=idx + dec + merge + append)
 
 
-def workload_config(w, num_splits: int, world: int) -> dict:
+def workload_config(w, num_splits: int, world: int, dcp: bool = False) -> dict:
     """The `config` object of the JSON line (both arms)."""
     kind, *a = w.ctx.split(":")
-    return {"workload": w.name, "description": w.description, "global_batch": w.batch * world,
+    par = "single GPU"
+    if world > 1:
+        par = f"decode context parallel x{world} (NCCL all-gather)" if dcp else f"replicas x{world}"
+    return {"workload": w.name, "description": w.description,
+            "global_batch": w.batch * (1 if dcp else world),
             "seq_len": int(a[-1]), "query_tokens": w.T, "kv_splits": num_splits,
             "topk_blocks": w.topk, "page_size": w.page_size,
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "parallelism": par,
             "l2": "inputs larger than L2 (2 GiB compressed keys read per step)",
             "timing": "value: K back-to-back steps (one CUDA graph of the K steps, replayed "
                       "once after an untimed replay; --no-graph: eager launches); kernel_ms and "
@@ -325,8 +333,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if args.batch is not None:
         from dataclasses import replace
         w = replace(w, batch=args.batch)
-    S = args.splits
-    batch = make_batch(w, dev, seed=rank_seed(w.seed, rank))
+    dcp = args.dcp and world > 1
+    S = world if dcp else args.splits
+    # replicas draw independent batches; DCP ranks share one batch
+    batch = make_batch(w, dev, seed=w.seed if dcp else rank_seed(w.seed, rank))
     B, T = w.batch, w.T
     L_host = batch.ctx_lens_host
     max_blocks = int((L_host.max() + 3) // 4)
@@ -351,6 +361,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     n_sel = ((L_host - T) // 4 + 1).to(torch.int32).to(dev) if T > 1 else None
     step = QSADecodeStep(cache, B, T, w.Hq, w.topk, S, max_blocks)
     stream = torch.cuda.current_stream()
+    dcp_step = None
+    if dcp:
+        from sparse_attention_decode_compress_b200.dcp import DCPDecode
+        dcp_step = DCPDecode(cache, B, T, w.Hq, w.topk)
 
     def one_step(ev=None):
         qapi.qsa_compress_append(cache, pos0, cu_new, k_new, T)
@@ -360,6 +374,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                             step.sel, None, step.ws_topk)
         if ev is not None:
             ev[1].record(stream)
+        if dcp_step is not None:  # this rank's split, all-gather, merge
+            dcp_step(batch.q, batch.ctx_lens, step.sel)
+            if ev is not None:
+                ev[2].record(stream)
+            return
         qapi.qsa_sparse_decode(cache, batch.q, batch.ctx_lens, step.sel, step.sm_scale, S,
                                step.o_part, step.lse_part, step.ws_dec)
         if ev is not None:
@@ -383,7 +402,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # graph holding the K steps (replayed once untimed first), or as eager
     # launches with --no-graph
     graph = None
-    if not args.no_graph:
+    if not args.no_graph and not dcp:  # (DCP steps hold collectives: eager)
         cap = torch.cuda.Stream()
         cap.wait_stream(stream)
         graph = torch.cuda.CUDAGraph()
@@ -434,7 +453,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # (qsa_session_*) uploads each step's inputs from pinned host memory and
     # downloads o / lse, overlapping the copies with the neighbouring steps
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not dcp:
         from sparse_attention_decode_compress_b200 import QSASession
         pin = lambda t: t.cpu().pin_memory()
         h_in = dict(pos0=pin(pos0), cu_new=pin(cu_new), k_new=pin(k_new), q_idx=pin(batch.q_idx),
@@ -486,15 +505,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     tot_bytes = sum(a["total"] for a in ab)
     peaks = measured_peaks()
     queries_per_step = B * T
-    value = weak_scaling_rate(queries_per_step, world, K, ms)
+    # replicas: every rank runs its own batch; DCP: the ranks share one batch
+    value = (weak_scaling_rate(queries_per_step, world, K, ms) if not dcp
+             else queries_per_step * K / (ms / 1e3))
     hbm = (tot_bytes * K / (ms / 1e3)) / 1e9
     achieved = idx_bytes / (topk_ms / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": w.kv_dtype if w.kv_dtype != "f32" else "f32",
+        "scaling": "strong" if dcp else "weak", "vs_baseline": None,
+        "dtype": w.kv_dtype if w.kv_dtype != "f32" else "f32",
         "data": "synthetic (seeded; stands in for the pages' 256k-context serving trace)",
-        "config": workload_config(w, S, world),
+        "config": workload_config(w, S, world, dcp),
         "hbm_gbs": round(hbm, 1),
         "hbm_pct_of_peak": round(100 * hbm / peaks["hbm_gbs"], 2),
         "hbm_pct_of_nominal_8tbs": round(100 * hbm / 8000.0, 2),

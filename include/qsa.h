@@ -234,6 +234,36 @@ qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32
                              void *workspace, size_t workspace_bytes, qsa_stream_t stream);
 
 /*
+ * qsa_sparse_decode_splits — qsa_sparse_decode for the splits
+ * [split_lo, split_hi) of num_splits only: what one rank of decode context
+ * parallelism computes when it holds one slice of the KV pages.
+ *
+ * Passage: blog "拉取请求实际改变了什么" (each decode-context-parallel rank
+ * reads its own slice of the cache; the partial results are merged at the
+ * end).
+ *
+ * Split s still owns logical pages [floor(s*NP/S), floor((s+1)*NP/S)) of
+ * S = num_splits. Pages outside the computed splits are never read, so the
+ * block table may leave them unmapped (-1).
+ *   o_part   [split_hi - split_lo, B, T, Hq, D] float32: split split_lo + i
+ *            in o_part[i]
+ *   lse_part [split_hi - split_lo, B, T, Hq] float32
+ *   0 <= split_lo < split_hi <= num_splits
+ *   other arguments as for qsa_sparse_decode (same workspace size for
+ *   num_splits)
+ * The computed splits are bit-identical to the same splits of a
+ * qsa_sparse_decode call with the same arguments.
+ * Errors: as qsa_sparse_decode; QSA_ERR_INVALID_ARG for an empty or
+ * out-of-range split range.
+ */
+qsa_status qsa_sparse_decode_splits(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
+                                    const void *q, int32_t q_dtype, const int32_t *ctx_lens,
+                                    const int32_t *sel, int32_t topk, float sm_scale,
+                                    int32_t num_splits, int32_t split_lo, int32_t split_hi,
+                                    float *o_part, float *lse_part, void *workspace,
+                                    size_t workspace_bytes, qsa_stream_t stream);
+
+/*
  * qsa_lse_merge — merge KV-partition partial results by log-sum-exp.
  *
  * Passage: blog "拉取请求实际改变了什么" (attention results from the ranks

@@ -3,12 +3,15 @@ hand-written sm_100a kernels (libqsa.so) and its thin PyTorch binding."""
 from .api import (QSACache, QSAError, QSASession, new_workspace, qsa_compress_append,
                   qsa_get_device_error, qsa_index_topk, qsa_index_topk_noalloc,
                   qsa_index_topk_tokens, qsa_index_topk_workspace_bytes, qsa_lse_merge,
-                  qsa_sparse_decode, qsa_sparse_decode_workspace_bytes)
+                  qsa_sparse_decode, qsa_sparse_decode_splits,
+                  qsa_sparse_decode_workspace_bytes)
+from .dcp import DCPDecode, dcp_exchange
 from .decode import QSADecodeStep
 
 __all__ = [
-    "QSACache", "QSAError", "QSADecodeStep", "QSASession", "new_workspace", "qsa_compress_append",
+    "DCPDecode", "QSACache", "QSAError", "QSADecodeStep", "QSASession", "dcp_exchange",
+    "new_workspace", "qsa_compress_append",
     "qsa_get_device_error", "qsa_index_topk", "qsa_index_topk_noalloc", "qsa_index_topk_tokens",
     "qsa_index_topk_workspace_bytes", "qsa_lse_merge",
-    "qsa_sparse_decode", "qsa_sparse_decode_workspace_bytes",
+    "qsa_sparse_decode", "qsa_sparse_decode_splits", "qsa_sparse_decode_workspace_bytes",
 ]

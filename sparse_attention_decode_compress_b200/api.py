@@ -223,6 +223,35 @@ def qsa_sparse_decode(cache: QSACache, q: torch.Tensor, ctx_lens: torch.Tensor,
            "qsa_sparse_decode")
 
 
+def qsa_sparse_decode_splits(cache: QSACache, q: torch.Tensor, ctx_lens: torch.Tensor,
+                             sel: torch.Tensor, sm_scale: float, num_splits: int, split_lo: int,
+                             split_hi: int, o_part: torch.Tensor, lse_part: torch.Tensor,
+                             workspace: torch.Tensor, stream=None) -> None:
+    """Splits [split_lo, split_hi) of num_splits only; o_part / lse_part
+    hold them from index 0 ([split_hi - split_lo, ...])."""
+    B, T, Hq, D = q.shape
+    q_dt = {torch.float32: _lib.QSA_F32, torch.bfloat16: _lib.QSA_BF16}.get(q.dtype)
+    if q_dt is None:
+        raise TypeError("q must be float32 or bfloat16")
+    _need(ctx_lens, torch.int32, "ctx_lens")
+    _need(sel, torch.int32, "sel")
+    _need(o_part, torch.float32, "o_part")
+    _need(lse_part, torch.float32, "lse_part")
+    n = split_hi - split_lo
+    if o_part.shape != (n, B, T, Hq, D) or lse_part.shape != (n, B, T, Hq):
+        raise ValueError("o_part must be [split_hi - split_lo, B, T, Hq, D] and lse_part "
+                         "[split_hi - split_lo, B, T, Hq]")
+    s = cache.struct()
+    lib = _lib.load()
+    _check(lib.qsa_sparse_decode_splits(ctypes.byref(s), B, T, Hq, _ptr(q), q_dt, _ptr(ctx_lens),
+                                        _ptr(sel), sel.shape[1], float(sm_scale), int(num_splits),
+                                        int(split_lo), int(split_hi), _ptr(o_part), _ptr(lse_part),
+                                        _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)),
+           "qsa_sparse_decode_splits")
+
+
 def qsa_lse_merge(o_part: torch.Tensor, lse_part: torch.Tensor, o: torch.Tensor,
                   lse: torch.Tensor, stream=None) -> None:
     for t, n in ((o_part, "o_part"), (lse_part, "lse_part"), (o, "o"), (lse, "lse")):

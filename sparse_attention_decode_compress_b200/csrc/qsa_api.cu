@@ -170,9 +170,10 @@ int decode_chunk_slots(int topk, int S, int chunk) {
 // more pairs than workers takes the largest chunks.  (Two or three smaller
 // chunks per warp, balanced through the work counter, measured ~30% slower:
 // each chunk's fixed plan / metadata / epilogue latency is paid again.)
-int decode_chunk_blocks(int B, int Hkv, int topk, int S, long long workers, int cap) {
+int decode_chunk_blocks(int B, int Hkv, int topk, int S, int S_active, long long workers,
+                        int cap) {
   const long long pairs = (long long)B * Hkv;
-  const long long per_split = workers / (pairs > 0 ? pairs : 1) / S;
+  const long long per_split = workers / (pairs > 0 ? pairs : 1) / S_active;
   int chunk = cap;
   if (per_split > 0) {
     const long long share = ((long long)topk + 2) * 6 / (5 * S);  // split share with 20% headroom
@@ -226,7 +227,8 @@ qsa_status launch_decode_warp(qsa::dec::Params p, cudaStream_t stream) {
   }
   const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
   const int ctas = bps * sm_count(dev);
-  p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, (long long)ctas * NW,
+  p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, p.s_hi - p.s_lo,
+                                (long long)ctas * NW,
                                 qsa::dec::kChunkBlocks);
   p.nch = decode_chunk_slots(p.topk, p.S, p.chunk);
   return launch(true, kernel, dim3(ctas), dim3(NW * 32), smem, stream, p);
@@ -270,7 +272,8 @@ qsa_status launch_decode_group(qsa::dec::Params p, cudaStream_t stream) {
   }
   const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
   const int ctas = bps * sm_count(dev);
-  p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, (long long)ctas * (NW / GW),
+  p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, p.s_hi - p.s_lo,
+                                (long long)ctas * (NW / GW),
                                 qsa::dec::kGroupChunkBlocks);
   p.nch = decode_chunk_slots(p.topk, p.S, p.chunk);
   return launch(true, kernel, dim3(ctas), dim3(NW * 32), smem, stream, p);
@@ -430,17 +433,24 @@ size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32
   return kTicketBytes + align_up(slots * M * D * sizeof(float)) + align_up(slots * M * sizeof(float));
 }
 
-qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
-                             const void *q, int32_t q_dtype, const int32_t *ctx_lens,
-                             const int32_t *sel, int32_t topk, float sm_scale,
-                             int32_t num_splits, float *o_part, float *lse_part,
-                             void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of qsa_sparse_decode and qsa_sparse_decode_splits: splits
+// [split_lo, split_hi) of num_splits, stored from o_part[0] on.
+qsa_status sparse_decode_call(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
+                              const void *q, int32_t q_dtype, const int32_t *ctx_lens,
+                              const int32_t *sel, int32_t topk, float sm_scale, int32_t num_splits,
+                              int32_t split_lo, int32_t split_hi, float *o_part, float *lse_part,
+                              void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
   qsa_status st = check_cache(cache);
   if (st != QSA_OK) return st;
   const int Hkv = cache->num_kv_heads;
   const int D = cache->head_dim;
   if (B < 0 || T < 1 || Hq < 1 || topk < 1 || topk > qsa::topk::kMaxTopk) return QSA_ERR_INVALID_ARG;
   if (num_splits < 1 || num_splits > qsa::dec::kMaxSplits) return QSA_ERR_INVALID_ARG;
+  if (split_lo < 0 || split_hi > num_splits || split_lo >= split_hi) return QSA_ERR_INVALID_ARG;
   if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return QSA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return QSA_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
@@ -488,6 +498,8 @@ qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32
   p.S = num_splits;
   p.o_part = o_part;
   p.lse_part = lse_part;
+  p.s_lo = split_lo;
+  p.s_hi = split_hi;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   p.counters = reinterpret_cast<int32_t *>(ws);
   p.tickets = p.counters + qsa::dec::kCounterInts;
@@ -499,6 +511,30 @@ qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (D == 64) return dispatch_decode_d<64>(p, cache->kv_dtype, s);
   return dispatch_decode_d<128>(p, cache->kv_dtype, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
+                             const void *q, int32_t q_dtype, const int32_t *ctx_lens,
+                             const int32_t *sel, int32_t topk, float sm_scale,
+                             int32_t num_splits, float *o_part, float *lse_part,
+                             void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
+  return sparse_decode_call(cache, B, T, Hq, q, q_dtype, ctx_lens, sel, topk, sm_scale, num_splits,
+                            0, num_splits, o_part, lse_part, workspace, workspace_bytes, stream);
+}
+
+qsa_status qsa_sparse_decode_splits(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
+                                    const void *q, int32_t q_dtype, const int32_t *ctx_lens,
+                                    const int32_t *sel, int32_t topk, float sm_scale,
+                                    int32_t num_splits, int32_t split_lo, int32_t split_hi,
+                                    float *o_part, float *lse_part, void *workspace,
+                                    size_t workspace_bytes, qsa_stream_t stream) {
+  return sparse_decode_call(cache, B, T, Hq, q, q_dtype, ctx_lens, sel, topk, sm_scale, num_splits,
+                            split_lo, split_hi, o_part, lse_part, workspace, workspace_bytes,
+                            stream);
 }
 
 qsa_status qsa_lse_merge(int32_t num_splits, int64_t rows, int32_t D, const float *o_part,

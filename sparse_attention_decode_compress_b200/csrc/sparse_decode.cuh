@@ -60,6 +60,9 @@ struct Params {
   int32_t *counters; // work counters of the persistent kernel (zero between calls)
   int nch;           // chunk slots per (r, g)
   int chunk;         // target micro-blocks per chunk, kMinChunkBlocks..kChunkBlocks
+  // splits computed: [s_lo, s_hi) of S (a decode-context-parallel rank
+  // computes its own); o_part / lse_part hold them from index 0
+  int s_lo = 0, s_hi = 0;
 };
 
 // Per-CTA plan, computed by warp 0.
@@ -168,7 +171,8 @@ __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl, int *stas
     pl.active = 0;
     for (int s = 0; s < p.S; ++s) {
       const int n = pl.e_bound[s + 1] - pl.e_bound[s];
-      const int ch = (n + p.chunk - 1) / p.chunk;  // chunks of n / ch <= p.chunk entries
+      // chunks of n / ch <= p.chunk entries; -1 marks a split not computed here
+      const int ch = (s < p.s_lo || s >= p.s_hi) ? -1 : (n + p.chunk - 1) / p.chunk;
       pl.ch_count[s] = ch;
       if (!pl.active && chunk >= cum && chunk < cum + ch) {
         const int k = chunk - cum;
@@ -180,16 +184,17 @@ __device__ void make_plan(const Params &p, int r, int chunk, Plan &pl, int *stas
         pl.e_begin = pl.e_bound[s] + (int)((long long)k * n / ch);
         pl.e_end = pl.e_bound[s] + (int)((long long)(k + 1) * n / ch);
       }
-      cum += ch;
+      cum += max(ch, 0);
     }
   }
   __syncwarp();
 }
 
-// Output row m of (r, g): query token t = m / G, head h = g*G + m % G.
+// Output row m of (r, g) in split s: query token t = m / G, head
+// h = g*G + m % G; splits are stored from s_lo on.
 __device__ __forceinline__ long long out_row(const Params &p, int s, int r, int g, int m) {
   const int t = m / p.G, h = g * p.G + m % p.G;
-  return (((long long)s * p.B + r) * p.T + t) * p.Hq + h;
+  return (((long long)(s - p.s_lo) * p.B + r) * p.T + t) * p.Hq + h;
 }
 
 // Empty splits of (r, g) get o = 0, lse = -inf (written by chunk 0's CTA).

@@ -1,0 +1,70 @@
+"""GPU checks of the decode-context-parallel split range: each split computed
+alone (qsa_sparse_decode_splits, as one DCP rank would) is bit-identical to
+the same split of a full qsa_sparse_decode, and merging the per-rank splits
+gives the step's output."""
+import numpy as np
+import pytest
+import torch
+
+import qsa_harness as H
+from sparse_attention_decode_compress_b200 import api
+from workloads.qsa_inputs import WORKLOADS, make_batch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _cuda_and_cleanup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name,lens,S", [("b32_32k", [9000, 12345, 4099], 2),
+                                         ("b128_256k", [40000, 30001], 4),
+                                         ("mtp_verify", [16384 + 3, 9001], 2),
+                                         ("mixed_fp8", [4096, 30007], 4)])
+def test_split_ranges_match_full_decode(name, lens, S):
+    b = make_batch(WORKLOADS[name], "cuda", ctx_lens=lens, seed=8)
+    w = b.w
+    step, cache = H.run_gpu(b, S, keep_scores=False)
+    Hkv, D = b.k_cache.shape[2], b.k_cache.shape[3]
+    ranges = [(s, s + 1) for s in range(S)] + ([(1, 3)] if S >= 3 else [])
+    o_parts, l_parts = [], []
+    for lo, hi in ranges:
+        ws = api.new_workspace(api.qsa_sparse_decode_workspace_bytes(w.batch, w.T, w.Hq, Hkv, D,
+                                                                     w.topk, S), "cuda")
+        o = torch.full((hi - lo,) + tuple(step.o_part.shape[1:]), 7.0, device="cuda")
+        l = torch.full((hi - lo,) + tuple(step.lse_part.shape[1:]), 7.0, device="cuda")
+        api.qsa_sparse_decode_splits(cache, b.q, b.ctx_lens, step.sel, step.sm_scale, S, lo, hi,
+                                     o, l, ws)
+        st, flags = api.qsa_get_device_error()
+        assert st == 0, (st, flags)
+        assert torch.equal(o, step.o_part[lo:hi]), (lo, hi)
+        assert torch.equal(l, step.lse_part[lo:hi]), (lo, hi)
+        if hi - lo == 1:
+            o_parts.append(o)
+            l_parts.append(l)
+    # what the ranks gather, merged
+    o_all, l_all = torch.cat(o_parts), torch.cat(l_parts)
+    o_m, l_m = torch.empty_like(step.o), torch.empty_like(step.lse)
+    api.qsa_lse_merge(o_all, l_all, o_m, l_m)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(o_m.cpu().numpy(), step.o.cpu().numpy())
+    np.testing.assert_array_equal(l_m.cpu().numpy(), step.lse.cpu().numpy())
+
+
+def test_split_range_rejected_on_host():
+    b = make_batch(WORKLOADS["b32_32k"], "cuda", ctx_lens=[5000], seed=2)
+    w = b.w
+    step, cache = H.run_gpu(b, 2, keep_scores=False)
+    ws = api.new_workspace(1 << 24, "cuda")
+    for lo, hi in ((1, 1), (-1, 1), (1, 3)):
+        n = max(hi - lo, 1)
+        o = torch.empty((n,) + tuple(step.o_part.shape[1:]), device="cuda")
+        l = torch.empty((n,) + tuple(step.lse_part.shape[1:]), device="cuda")
+        with pytest.raises((api.QSAError, ValueError)):
+            api.qsa_sparse_decode_splits(cache, b.q, b.ctx_lens, step.sel, step.sm_scale, 2, lo, hi,
+                                         o, l, ws)

@@ -42,12 +42,14 @@ def _worker(rank, world, port, q):
         V = rng.standard_normal((L, Hkv, D))
         toks = np.sort(rng.choice(L, 300, replace=False))
         o_part, lse_part = ref.split_attention(qv, K, V, toks, 0.25, L, P, world)
-        mine = torch.from_numpy(np.concatenate([o_part[rank].ravel(), lse_part[rank]]))
-        got = [torch.empty_like(mine) for _ in range(world)]
-        dist.all_gather(got, mine)
-        o_g = np.stack([g[:Hq * D].numpy().reshape(Hq, D) for g in got])
-        l_g = np.stack([g[Hq * D:].numpy() for g in got])
-        o_m, lse_m = ref.lse_merge(o_g, l_g)
+        # the library's exchange: this rank's split in, every rank's out
+        from sparse_attention_decode_compress_b200.dcp import dcp_exchange
+        o_loc = torch.from_numpy(o_part[rank][None].copy())
+        l_loc = torch.from_numpy(lse_part[rank][None].copy())
+        o_all = torch.empty((world,) + o_loc.shape[1:], dtype=o_loc.dtype)
+        l_all = torch.empty((world,) + l_loc.shape[1:], dtype=l_loc.dtype)
+        dcp_exchange(o_loc, l_loc, o_all, l_all)
+        o_m, lse_m = ref.lse_merge(o_all.numpy(), l_all.numpy())
         o_u, lse_u = ref.attention(qv, K, V, toks, 0.25)
         out["dcp_err"] = float(max(np.abs(o_m - o_u).max(), np.abs(lse_m - lse_u).max()))
         q.put((rank, out))
