@@ -1,5 +1,5 @@
 // Shared device helpers of the QSA kernels (sm_100a): the per-device error
-// word, bounded mbarrier waits, bulk (TMA-engine) copies and cp.async.
+// word, programmatic launch, cp.async, named barriers and L2 policies.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -13,7 +13,7 @@ namespace qsa {
 // Error bits of the per-device error word (read by qsa_get_device_error).
 enum : uint32_t {
   kErrBounds = 1u,    // block-table entry / logical page / position out of range
-  kErrTimeout = 2u,   // a bounded wait ran out
+  kErrTimeout = 2u,   // a bounded wait ran out (kept for the ABI; no kernel of this version waits)
   kErrBadInput = 4u,  // malformed lengths, counts or selection rows
 };
 
@@ -37,102 +37,16 @@ __device__ __forceinline__ void pdl_open() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// A bounded wait gives up after about this many SM cycles (~1 s at 1.9 GHz).
-constexpr long long kWaitCycles = 2000000000LL;
-
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// ---------------------------------------------------------------- mbarrier --
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-               : "memory");
-}
-
-// Makes mbarrier initialisation visible to the async (bulk copy) proxy.
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  asm volatile(
-      "{\n\t.reg .b64 st;\n\t"
-      "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile(
-      "{\n\t.reg .b64 st;\n\t"
-      "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
-      "r"(bytes)
-      : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Waits for the phase with the given parity to complete.  Gives up after
-// kWaitCycles, records kErrTimeout and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) {
-      record_error(kErrTimeout);
-      return false;
-    }
-  }
-  return true;
-}
-
-// Same, but shares a CTA-wide abort flag: once any thread of the CTA has
-// given up, every later wait returns false at once (so a stalled pipeline
-// costs one timeout, not one per stage).
-__device__ __forceinline__ bool mbar_wait_abortable(uint64_t *bar, uint32_t parity,
-                                                    volatile int *abort_flag) {
-  if (*abort_flag) return false;
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
-      record_error(kErrTimeout);
-      *abort_flag = 1;
-      return false;
-    }
-  }
-  return true;
-}
-
-// -------------------------------------------------------------- bulk copy --
-// L2 policy: streamed data that is read once.
+// ------------------------------------------------------------- L2 policy --
+// Streamed data that is read once.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
-}
-
-// Global -> shared bulk copy completed on `bar` (complete_tx).  dst, src and
-// bytes must be multiples of 16.
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
-                                         uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
 }
 
 // --------------------------------------------------------------- cp.async --
@@ -162,31 +76,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ long long ceil_div_ll(long long a, long long b) {
   return (a + b - 1) / b;
-}
-
-__device__ __forceinline__ int ld_cg_s32(const int32_t *p) {
-  int v;
-  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ int4 ld_cg_v4(const int32_t *p) {
-  int4 v;
-  asm volatile("ld.global.cg.v4.s32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-__device__ __forceinline__ float4 ld_cg_f4(const float *p) {
-  float4 v;
-  asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "l"(p));
-  return v;
-}
-__device__ __forceinline__ float ld_cg_f32(const float *p) {
-  float v;
-  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
-  return v;
 }
 
 // Cache description passed to kernels by value.
