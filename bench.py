@@ -525,7 +525,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      "peak_source": peaks["source"], "traffic": index_topk_traffic(B),
                      "launch_ms": round(topk_ms, 5), "algorithmic_bytes_per_launch": idx_bytes},
         "kernel_ms": {"index_topk": round(topk_ms, 5), "sparse_decode": round(dec_ms, 5)},
-        "gpu_launches": QSADecodeStep.KERNELS_PER_STEP * K,
+        "gpu_launches": step.kernels_per_step * K,
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -234,6 +234,29 @@ qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32
                              void *workspace, size_t workspace_bytes, qsa_stream_t stream);
 
 /*
+ * qsa_sparse_decode_merged — qsa_sparse_decode followed by the split merge
+ * (qsa_lse_merge of o_part / lse_part into o / lse), in one call: the two
+ * kernels go back to back on the stream.
+ *
+ * Passage: as qsa_sparse_decode and qsa_lse_merge (blog "拉取请求实际改变了
+ * 什么": partial results of the context slices are merged at the end).
+ *
+ *   o    [B, T, Hq, D] float32 output, 16-byte aligned
+ *   lse  [B, T, Hq] float32 output
+ *   other arguments as for qsa_sparse_decode; o_part / lse_part are still
+ *   written (same values as qsa_sparse_decode)
+ * o / lse are those of qsa_lse_merge(num_splits, B*T*Hq, D, o_part,
+ * lse_part, o, lse).
+ * Errors: as qsa_sparse_decode and qsa_lse_merge.
+ */
+qsa_status qsa_sparse_decode_merged(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
+                                    const void *q, int32_t q_dtype, const int32_t *ctx_lens,
+                                    const int32_t *sel, int32_t topk, float sm_scale,
+                                    int32_t num_splits, float *o_part, float *lse_part, float *o,
+                                    float *lse, void *workspace, size_t workspace_bytes,
+                                    qsa_stream_t stream);
+
+/*
  * qsa_sparse_decode_splits — qsa_sparse_decode for the splits
  * [split_lo, split_hi) of num_splits only: what one rank of decode context
  * parallelism computes when it holds one slice of the KV pages.
@@ -327,8 +350,8 @@ qsa_status qsa_get_device_error(qsa_stream_t stream, uint32_t *flags_out);
  * - Its upload stream copies step k+1's inputs while step k computes on the
  *   compute stream, and its download stream copies step k-1's o / lse back.
  *   Events order the three streams.
- * - A step runs exactly qsa_compress_append, qsa_index_topk,
- *   qsa_sparse_decode (sm_scale, num_splits) and qsa_lse_merge.
+ * - A step runs exactly qsa_compress_append, qsa_index_topk and
+ *   qsa_sparse_decode_merged (sm_scale, num_splits).
  *
  * qsa_session_create allocates every buffer (cudaMalloc, the decode
  * workspace zero-filled) and two non-blocking streams. It copies *cache

@@ -3,7 +3,7 @@ hand-written sm_100a kernels (libqsa.so) and its thin PyTorch binding."""
 from .api import (QSACache, QSAError, QSASession, new_workspace, qsa_compress_append,
                   qsa_get_device_error, qsa_index_topk, qsa_index_topk_noalloc,
                   qsa_index_topk_tokens, qsa_index_topk_workspace_bytes, qsa_lse_merge,
-                  qsa_sparse_decode, qsa_sparse_decode_splits,
+                  qsa_sparse_decode, qsa_sparse_decode_merged, qsa_sparse_decode_splits,
                   qsa_sparse_decode_workspace_bytes)
 from .dcp import DCPDecode, dcp_exchange
 from .decode import QSADecodeStep
@@ -13,5 +13,6 @@ __all__ = [
     "new_workspace", "qsa_compress_append",
     "qsa_get_device_error", "qsa_index_topk", "qsa_index_topk_noalloc", "qsa_index_topk_tokens",
     "qsa_index_topk_workspace_bytes", "qsa_lse_merge",
-    "qsa_sparse_decode", "qsa_sparse_decode_splits", "qsa_sparse_decode_workspace_bytes",
+    "qsa_sparse_decode", "qsa_sparse_decode_merged", "qsa_sparse_decode_splits",
+    "qsa_sparse_decode_workspace_bytes",
 ]

@@ -38,6 +38,10 @@ SIGNATURES = {
     "qsa_sparse_decode": (c_int32, [ctypes.POINTER(QsaCacheStruct), c_int32, c_int32, c_int32,
                                     c_void_p, c_int32, c_void_p, c_void_p, c_int32, c_float,
                                     c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qsa_sparse_decode_merged": (c_int32, [ctypes.POINTER(QsaCacheStruct), c_int32, c_int32, c_int32,
+                                           c_void_p, c_int32, c_void_p, c_void_p, c_int32, c_float,
+                                           c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                           c_size_t, c_void_p]),
     "qsa_sparse_decode_splits": (c_int32, [ctypes.POINTER(QsaCacheStruct), c_int32, c_int32, c_int32,
                                            c_void_p, c_int32, c_void_p, c_void_p, c_int32, c_float,
                                            c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p,

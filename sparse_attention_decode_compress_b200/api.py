@@ -223,6 +223,35 @@ def qsa_sparse_decode(cache: QSACache, q: torch.Tensor, ctx_lens: torch.Tensor,
            "qsa_sparse_decode")
 
 
+def qsa_sparse_decode_merged(cache: QSACache, q: torch.Tensor, ctx_lens: torch.Tensor,
+                             sel: torch.Tensor, sm_scale: float, num_splits: int,
+                             o_part: torch.Tensor, lse_part: torch.Tensor, o: torch.Tensor,
+                             lse: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    """qsa_sparse_decode and the split merge in one call (o / lse as
+    qsa_lse_merge of o_part / lse_part; two kernels)."""
+    B, T, Hq, D = q.shape
+    q_dt = {torch.float32: _lib.QSA_F32, torch.bfloat16: _lib.QSA_BF16}.get(q.dtype)
+    if q_dt is None:
+        raise TypeError("q must be float32 or bfloat16")
+    for t, n in ((o_part, "o_part"), (lse_part, "lse_part"), (o, "o"), (lse, "lse")):
+        _need(t, torch.float32, n)
+    _need(ctx_lens, torch.int32, "ctx_lens")
+    _need(sel, torch.int32, "sel")
+    if o_part.shape != (num_splits, B, T, Hq, D) or lse_part.shape != (num_splits, B, T, Hq):
+        raise ValueError("o_part must be [S, B, T, Hq, D] and lse_part [S, B, T, Hq]")
+    if o.shape != (B, T, Hq, D) or lse.shape != (B, T, Hq):
+        raise ValueError("o must be [B, T, Hq, D] and lse [B, T, Hq]")
+    s = cache.struct()
+    lib = _lib.load()
+    _check(lib.qsa_sparse_decode_merged(ctypes.byref(s), B, T, Hq, _ptr(q), q_dt, _ptr(ctx_lens),
+                                        _ptr(sel), sel.shape[1], float(sm_scale), int(num_splits),
+                                        _ptr(o_part), _ptr(lse_part), _ptr(o), _ptr(lse),
+                                        _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)),
+           "qsa_sparse_decode_merged")
+
+
 def qsa_sparse_decode_splits(cache: QSACache, q: torch.Tensor, ctx_lens: torch.Tensor,
                              sel: torch.Tensor, sm_scale: float, num_splits: int, split_lo: int,
                              split_hi: int, o_part: torch.Tensor, lse_part: torch.Tensor,

@@ -443,7 +443,8 @@ qsa_status sparse_decode_call(const qsa_cache *cache, int32_t B, int32_t T, int3
                               const void *q, int32_t q_dtype, const int32_t *ctx_lens,
                               const int32_t *sel, int32_t topk, float sm_scale, int32_t num_splits,
                               int32_t split_lo, int32_t split_hi, float *o_part, float *lse_part,
-                              void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
+                              float *o_merged, float *lse_merged, void *workspace,
+                              size_t workspace_bytes, qsa_stream_t stream) {
   qsa_status st = check_cache(cache);
   if (st != QSA_OK) return st;
   const int Hkv = cache->num_kv_heads;
@@ -470,6 +471,9 @@ qsa_status sparse_decode_call(const qsa_cache *cache, int32_t B, int32_t T, int3
   if ((size_t)B * Hkv * num_splits * sizeof(int32_t) >
       kTicketBytes - qsa::dec::kCounterInts * sizeof(int32_t))
     return QSA_ERR_UNSUPPORTED;
+  const bool merged = o_merged != nullptr;
+  if (merged && (!lse_merged || !aligned(o_merged, 16) || split_lo != 0 || split_hi != num_splits))
+    return QSA_ERR_INVALID_ARG;
   if (!q || !ctx_lens || !sel || !o_part || !lse_part || !workspace || !cache->k_cache ||
       !cache->v_cache)
     return QSA_ERR_INVALID_ARG;
@@ -503,14 +507,22 @@ qsa_status sparse_decode_call(const qsa_cache *cache, int32_t B, int32_t T, int3
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   p.counters = reinterpret_cast<int32_t *>(ws);
   p.tickets = p.counters + qsa::dec::kCounterInts;
+
   const size_t slots = (size_t)B * Hkv * nch;
   p.ws_o = reinterpret_cast<float *>(ws + kTicketBytes);
   p.ws_lse = reinterpret_cast<float *>(ws + kTicketBytes + align_up(slots * M * D * sizeof(float)));
   p.nch = nch;  // the launch sets nch and chunk for its kernel
   p.chunk = qsa::dec::kMinChunkBlocks;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (D == 64) return dispatch_decode_d<64>(p, cache->kv_dtype, s);
-  return dispatch_decode_d<128>(p, cache->kv_dtype, s);
+  st = (D == 64) ? dispatch_decode_d<64>(p, cache->kv_dtype, s)
+                 : dispatch_decode_d<128>(p, cache->kv_dtype, s);
+  // the merge kernel, one warp per output row, right behind the decode
+  // (merging inside the decode, by the warp finishing a pair's last split,
+  // measured slower: 0.434 against 0.423 ms per 256k step, 0.228 against
+  // 0.176 ms per MTP step, from the one warp walking all of a pair's rows)
+  if (st != QSA_OK || !merged) return st;
+  return qsa_lse_merge(num_splits, (int64_t)B * T * Hq, D, o_part, lse_part, o_merged, lse_merged,
+                       stream);
 }
 
 }  // namespace
@@ -523,7 +535,20 @@ qsa_status qsa_sparse_decode(const qsa_cache *cache, int32_t B, int32_t T, int32
                              int32_t num_splits, float *o_part, float *lse_part,
                              void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
   return sparse_decode_call(cache, B, T, Hq, q, q_dtype, ctx_lens, sel, topk, sm_scale, num_splits,
-                            0, num_splits, o_part, lse_part, workspace, workspace_bytes, stream);
+                            0, num_splits, o_part, lse_part, nullptr, nullptr, workspace,
+                            workspace_bytes, stream);
+}
+
+qsa_status qsa_sparse_decode_merged(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
+                                    const void *q, int32_t q_dtype, const int32_t *ctx_lens,
+                                    const int32_t *sel, int32_t topk, float sm_scale,
+                                    int32_t num_splits, float *o_part, float *lse_part, float *o,
+                                    float *lse, void *workspace, size_t workspace_bytes,
+                                    qsa_stream_t stream) {
+  if (B > 0 && (!o || !lse)) return QSA_ERR_INVALID_ARG;
+  return sparse_decode_call(cache, B, T, Hq, q, q_dtype, ctx_lens, sel, topk, sm_scale, num_splits,
+                            0, num_splits, o_part, lse_part, o, lse, workspace, workspace_bytes,
+                            stream);
 }
 
 qsa_status qsa_sparse_decode_splits(const qsa_cache *cache, int32_t B, int32_t T, int32_t Hq,
@@ -533,8 +558,8 @@ qsa_status qsa_sparse_decode_splits(const qsa_cache *cache, int32_t B, int32_t T
                                     float *o_part, float *lse_part, void *workspace,
                                     size_t workspace_bytes, qsa_stream_t stream) {
   return sparse_decode_call(cache, B, T, Hq, q, q_dtype, ctx_lens, sel, topk, sm_scale, num_splits,
-                            split_lo, split_hi, o_part, lse_part, workspace, workspace_bytes,
-                            stream);
+                            split_lo, split_hi, o_part, lse_part, nullptr, nullptr, workspace,
+                            workspace_bytes, stream);
 }
 
 qsa_status qsa_lse_merge(int32_t num_splits, int64_t rows, int32_t D, const float *o_part,

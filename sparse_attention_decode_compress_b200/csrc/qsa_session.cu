@@ -4,7 +4,8 @@
 // The session owns the device side of a decode loop: two slots of input and
 // output buffers, the selection, the split partials and both workspaces.  A
 // step copies its inputs host -> device on the session's upload stream,
-// runs the four library calls on the compute stream, and copies o and lse
+// runs qsa_compress_append, qsa_index_topk and qsa_sparse_decode_merged on
+// the compute stream, and copies o and lse
 // back on the download stream.  Slots alternate, so the upload of step k+1
 // and the download of step k-1 run while step k computes.  Events order the
 // three streams:
@@ -202,11 +203,9 @@ qsa_status qsa_session_step_host(qsa_session *s, const int32_t *pos0, const int3
     st = qsa_index_topk(&s->cache, B, s->q_idx[k], s->ctx_lens[k], n_sel ? s->n_sel[k] : nullptr,
                         s->max_blocks, s->topk, s->sel, nullptr, s->ws_topk, s->ws_topk_bytes, cs);
   if (st == QSA_OK)
-    st = qsa_sparse_decode(&s->cache, B, s->T, s->Hq, s->q[k], s->q_dtype, s->ctx_lens[k], s->sel,
-                           s->topk, s->sm_scale, s->S, s->o_part, s->lse_part, s->ws_dec,
-                           s->ws_dec_bytes, cs);
-  if (st == QSA_OK)
-    st = qsa_lse_merge(s->S, (int64_t)rows, s->D, s->o_part, s->lse_part, s->o[k], s->lse[k], cs);
+    st = qsa_sparse_decode_merged(&s->cache, B, s->T, s->Hq, s->q[k], s->q_dtype, s->ctx_lens[k],
+                                  s->sel, s->topk, s->sm_scale, s->S, s->o_part, s->lse_part,
+                                  s->o[k], s->lse[k], s->ws_dec, s->ws_dec_bytes, cs);
   if (st != QSA_OK) return st;
   // download once the step is computed
   ok = cudaEventRecord(s->compute_done[k], s->compute) == cudaSuccess;

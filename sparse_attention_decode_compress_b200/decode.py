@@ -1,6 +1,7 @@
 """One decode step of the QSA hot path through the C ABI:
-compress-append -> index top-k -> sparse split-KV decode -> LSE merge.
-Holds the step's output buffers and workspaces; every step is a kernel."""
+compress-append -> index top-k -> sparse split-KV decode and the LSE merge
+of its splits (qsa_sparse_decode_merged: two kernels).  Holds the step's output buffers
+and workspaces; every step is a kernel."""
 from __future__ import annotations
 
 import math
@@ -8,7 +9,7 @@ import math
 import torch
 
 from .api import (QSACache, new_workspace, qsa_compress_append, qsa_index_topk,
-                  qsa_index_topk_workspace_bytes, qsa_lse_merge, qsa_sparse_decode,
+                  qsa_index_topk_workspace_bytes, qsa_sparse_decode_merged,
                   qsa_sparse_decode_workspace_bytes)
 
 
@@ -35,10 +36,9 @@ class QSADecodeStep:
         qsa_compress_append(self.cache, pos0, cu_new, k_new, self.T, stream)
         qsa_index_topk(self.cache, q_idx, ctx_lens, n_sel, self.max_blocks, self.topk, self.sel,
                        self.scores, self.ws_topk, stream)
-        qsa_sparse_decode(self.cache, q, ctx_lens, self.sel, self.sm_scale, self.S, self.o_part,
-                          self.lse_part, self.ws_dec, stream)
-        qsa_lse_merge(self.o_part, self.lse_part, self.o, self.lse, stream)
+        qsa_sparse_decode_merged(self.cache, q, ctx_lens, self.sel, self.sm_scale, self.S,
+                                 self.o_part, self.lse_part, self.o, self.lse, self.ws_dec, stream)
         return self.o, self.lse
 
-    # kernels one call launches: append, scan + select, decode, merge
-    KERNELS_PER_STEP = 5
+    # kernels one call launches: append, scan, select, decode, merge
+    kernels_per_step = 5
