@@ -167,14 +167,17 @@ int decode_chunk_slots(int topk, int S, int chunk) {
 // floor(workers / pairs) workers, c = that / S per split; its splits hold
 // about (topk + 2) / S entries each, with 20% added for splits that hold
 // more than their share, so that each split takes c chunks.  A batch with
-// more pairs than workers takes the largest chunks.  (Two or three smaller
-// chunks per warp, balanced through the work counter, measured ~30% slower:
-// each chunk's fixed plan / metadata / epilogue latency is paid again.)
+// fewer workers than splits takes the largest chunks, and with
+// `whole_splits` (a kernel that streams an item in pieces) whole splits:
+// one item per split, no chunk merge.  (Two or three smaller chunks per
+// warp, balanced through the work counter, measured ~30% slower: each
+// chunk's fixed plan / metadata / epilogue latency is paid again.)
 int decode_chunk_blocks(int B, int Hkv, int topk, int S, int S_active, long long workers,
-                        int cap) {
+                        int cap, bool whole_splits) {
   const long long pairs = (long long)B * Hkv;
   const long long per_split = workers / (pairs > 0 ? pairs : 1) / S_active;
   int chunk = cap;
+  if (per_split == 0 && whole_splits) chunk = topk + 2;
   if (per_split > 0) {
     const long long share = ((long long)topk + 2) * 6 / (5 * S);  // split share with 20% headroom
     chunk = (int)std::min<long long>(chunk, (share + per_split - 1) / per_split);
@@ -229,7 +232,7 @@ qsa_status launch_decode_warp(qsa::dec::Params p, cudaStream_t stream) {
   const int ctas = bps * sm_count(dev);
   p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, p.s_hi - p.s_lo,
                                 (long long)ctas * NW,
-                                qsa::dec::kChunkBlocks);
+                                qsa::dec::warp_piece_blocks<FP8>(), true);
   p.nch = decode_chunk_slots(p.topk, p.S, p.chunk);
   return launch(true, kernel, dim3(ctas), dim3(NW * 32), smem, stream, p);
 }
@@ -250,11 +253,14 @@ qsa_status launch_decode_f32(qsa::dec::Params p, cudaStream_t stream) {
 }
 
 // More than 8 query rows: groups of GW = NT warps, one per 8-row tile,
-// sharing a ring of NS = 2 * GW stages (12 warps per SM).
+// sharing a ring of NS stages.  bf16: 16 warps per SM (4 groups of 4 at MTP
+// verify) with one stage per warp, 128 registers; fp8: 12 warps with two
+// stages per warp (at 16 warps its registers spill).  (MTP verify decode:
+// 16 warps x 1 stage 63.5 us, 16 x 1.5 65.3 us, 12 x 2 67.1 us.)
 template <int D, bool FP8, int GW>
 qsa_status launch_decode_group(qsa::dec::Params p, cudaStream_t stream) {
-  constexpr int NW = 12;
-  constexpr int NS = 2 * GW;
+  constexpr int NW = (FP8 ? 12 : 16) / GW * GW;
+  constexpr int NS = FP8 ? 2 * GW : GW;
   static bool done[kMaxDevices] = {false};
   static int blocks_per_sm[kMaxDevices] = {0};
   auto kernel = qsa::dec::sparse_decode_group_kernel<D, FP8, NW, NS, GW>;
@@ -274,7 +280,7 @@ qsa_status launch_decode_group(qsa::dec::Params p, cudaStream_t stream) {
   const int ctas = bps * sm_count(dev);
   p.chunk = decode_chunk_blocks(p.B, p.c.num_kv_heads, p.topk, p.S, p.s_hi - p.s_lo,
                                 (long long)ctas * (NW / GW),
-                                qsa::dec::kGroupChunkBlocks);
+                                qsa::dec::kGroupChunkBlocks, false);
   p.nch = decode_chunk_slots(p.topk, p.S, p.chunk);
   return launch(true, kernel, dim3(ctas), dim3(NW * 32), smem, stream, p);
 }

@@ -109,31 +109,9 @@ __device__ __forceinline__ void issue_stage_group(const Params &p, WS &W, int sl
     const int kv = it / (kTokW * kCh);
     const int rem = it % (kTokW * kCh);
     const int row = rem / kCh, ch = rem % kCh;
-    uint8_t *dst = W.ring[slot][kv] + (FP8 ? (row * kRowBytes + ch * 16) : swz<D>(row, ch));
+    uint8_t *dst = W.ring[slot][kv] + (FP8 ? fp8_swz<D>(row, ch) : swz<D>(row, ch));
     const uint8_t *src = (kv ? vbase : kbase) + (long long)off[i] * kRowBytes + ch * 16;
     cp_async16_zfill(dst, src, load[i]);
-  }
-}
-
-// FP8 -> bf16 conversion of one 16-token K or V stage, shared by a group.
-template <int D, int GW>
-__device__ __forceinline__ void convert_fp8_rows_group(const uint8_t *raw, uint8_t *dst, int tig) {
-  constexpr int kChunks = kTokW * D / 8;
-  for (int it = tig; it < kChunks; it += GW * 32) {
-    const int row = it / (D / 8), ch = it % (D / 8);
-    const uint2 v = *reinterpret_cast<const uint2 *>(raw + row * D + ch * 8);
-    const uint32_t w[2] = {v.x, v.y};
-    uint32_t outw[4];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const __nv_fp8x2_storage_t lo = (__nv_fp8x2_storage_t)(w[j] & 0xffffu);
-      const __nv_fp8x2_storage_t hi = (__nv_fp8x2_storage_t)(w[j] >> 16);
-      const float2 flo = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(lo, __NV_E4M3)));
-      const float2 fhi = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(hi, __NV_E4M3)));
-      outw[2 * j] = pack_bf16(flo.x, flo.y);
-      outw[2 * j + 1] = pack_bf16(fhi.x, fhi.y);
-    }
-    *reinterpret_cast<uint4 *>(dst + swz<D>(row, ch)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
   }
 }
 
@@ -177,18 +155,28 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
     const int g = (it / p.nch) % Hkv;
     const int r = it / (p.nch * Hkv);
 
-    // Q B-fragments of this warp's tile: rows m = 8 * wig + gq
+    // Q B-fragments of this warp's tile: rows m = 8 * wig + gq (fp8: f16
+    // in the order of fp8_frag.cuh); csc = the logit factor of each column
     uint32_t qb[MD][2];
+    float csc[2];
     {
       const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
       const int m = 8 * wig + gq;
       const bool ok = m < p.M;
       const __nv_bfloat16 *qrow =
           qg + (((long long)r * p.T + (ok ? m / p.G : 0)) * p.Hq + g * p.G + (ok ? m % p.G : 0)) * D;
+      if constexpr (FP8) {
+        const float qinv = q_frags_f16<D>(ok ? qrow : nullptr, cq, qb);
 #pragma unroll
-      for (int kk = 0; kk < MD; ++kk) {
-        qb[kk][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq) : 0u;
-        qb[kk][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq + 8) : 0u;
+        for (int e = 0; e < 2; ++e)
+          csc[e] = p.scale_log2 * __shfl_sync(0xffffffffu, qinv, (2 * cq + e) * 4);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < MD; ++kk) {
+          qb[kk][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq) : 0u;
+          qb[kk][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq + 8) : 0u;
+        }
+        csc[0] = csc[1] = p.scale_log2;
       }
     }
     constexpr int kStashInts = (int)(sizeof(W.ring[0]) / sizeof(int));
@@ -202,6 +190,8 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
     if (!pl.active) continue;
     fill_meta_group<WS, FP8>(p, pl, r, g, W, tig, GW * 32, stash);
     gsync();
+    const float vsref = FP8 ? chunk_vsref(W, pl.e_end - pl.e_begin, lane) : 1.f;
+    const float vsinv = 1.f / vsref;
 
     int tcol[2];
 #pragma unroll
@@ -228,30 +218,24 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
         cp_async_commit();
       }
       const int slot = st % NS;
-      const uint8_t *ks_t;
-      const uint8_t *vs_t;
-      if constexpr (FP8) {
-        convert_fp8_rows_group<D, GW>(W.ring[slot][0], W.cvt[0], tig);
-        convert_fp8_rows_group<D, GW>(W.ring[slot][1], W.cvt[1], tig);
-        gsync();
-        ks_t = W.cvt[0];
-        vs_t = W.cvt[1];
-      } else {
-        ks_t = W.ring[slot][0];
-        vs_t = W.ring[slot][1];
-      }
+      const uint8_t *ks_t = W.ring[slot][0];
+      const uint8_t *vs_t = W.ring[slot][1];
       const int tb = st * kTokW;
 
       // ---- S^T = K Q^T for this warp's tile
       float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sac2[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (FP8) {
+        qk_fp8<D>(ks_t, gq, cq, qb, sacc, sac2);
+      } else {
 #pragma unroll
-      for (int kk = 0; kk < MD; ++kk) {
-        uint32_t a0, a1, a2, a3;
-        const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int ch = 2 * kk + (lane >> 4);
-        ldsm_x4(a0, a1, a2, a3, ks_t + swz<D>(row, ch));
-        if (kk & 1) mma_bf16(sac2, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
-        else mma_bf16(sacc, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+        for (int kk = 0; kk < MD; ++kk) {
+          uint32_t a0, a1, a2, a3;
+          const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+          const int ch = 2 * kk + (lane >> 4);
+          ldsm_x4(a0, a1, a2, a3, ks_t + swz<D>(row, ch));
+          if (kk & 1) mma_bf16(sac2, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+          else mma_bf16(sacc, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+        }
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[e] += sac2[e];
@@ -262,8 +246,8 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
       if constexpr (FP8) {
         ksc0 = W.ks[(tb + gq) >> 2];
         ksc1 = W.ks[(tb + gq + 8) >> 2];
-        vsc0 = W.vs[(tb + gq) >> 2];
-        vsc1 = W.vs[(tb + gq + 8) >> 2];
+        vsc0 = W.vs[(tb + gq) >> 2] * vsinv;
+        vsc1 = W.vs[(tb + gq + 8) >> 2] * vsinv;
       }
       float x[4];
 #pragma unroll
@@ -271,8 +255,8 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
         const int t = tcol[e];
         const bool ok0 = t >= 0 && ((vm0 >> t) & 1u);
         const bool ok1 = t >= 0 && ((vm1 >> t) & 1u);
-        x[e] = ok0 ? sacc[e] * p.scale_log2 * ksc0 : -INFINITY;
-        x[2 + e] = ok1 ? sacc[2 + e] * p.scale_log2 * ksc1 : -INFINITY;
+        x[e] = ok0 ? sacc[e] * csc[e] * ksc0 : -INFINITY;
+        x[2 + e] = ok1 ? sacc[2 + e] * csc[e] * ksc1 : -INFINITY;
       }
       float pj[4], alpha[2];
       bool rescale = false;
@@ -294,13 +278,8 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
         lcol[e] = lcol[e] * a + pj[e] + pj[2 + e];
       }
       const float v0 = pj[0] * vsc0, v1 = pj[1] * vsc0, v2 = pj[2] * vsc1, v3 = pj[3] * vsc1;
-      const __nv_bfloat162 h01 = __floats2bfloat162_rn(v0, v1);
-      const __nv_bfloat162 h23 = __floats2bfloat162_rn(v2, v3);
-      const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
-      const uint32_t bhi0 = movmatrix_t(*reinterpret_cast<const uint32_t *>(&h01));
-      const uint32_t bhi1 = movmatrix_t(*reinterpret_cast<const uint32_t *>(&h23));
-      const uint32_t blo0 = movmatrix_t(pack_bf16(v0 - f01.x, v1 - f01.y));
-      const uint32_t blo1 = movmatrix_t(pack_bf16(v2 - f23.x, v3 - f23.y));
+      uint32_t bhi[2], blo[2];
+      p_frags<FP8>(v0, v1, v2, v3, bhi, blo);
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int i = 0; i < MD; ++i) {
@@ -312,14 +291,26 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
       }
 
       // ---- O^T += V^T P^T
+      if constexpr (FP8) {
+        VRaw<D> vr;
+        v_raw_fp8<D>(vs_t, gq, cq, vr);
 #pragma unroll
-      for (int i = 0; i < MD; ++i) {
-        uint32_t a0, a1, a2, a3;
-        const int row = (lane & 7) + 8 * (lane >> 4);
-        const int ch = 2 * i + ((lane >> 3) & 1);
-        ldsm_x4_t(a0, a1, a2, a3, vs_t + swz<D>(row, ch));
-        mma_bf16(o[i], a0, a1, a2, a3, bhi0, bhi1);
-        mma_bf16(o[i], a0, a1, a2, a3, blo0, blo1);
+        for (int i = 0; i < MD; ++i) {
+          uint32_t a0, a1, a2, a3;
+          v_frag_fp8<D>(vr, i, a0, a1, a2, a3);
+          mma_f16(o[i], a0, a1, a2, a3, bhi[0], bhi[1]);
+          mma_f16(o[i], a0, a1, a2, a3, blo[0], blo[1]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < MD; ++i) {
+          uint32_t a0, a1, a2, a3;
+          const int row = (lane & 7) + 8 * (lane >> 4);
+          const int ch = 2 * i + ((lane >> 3) & 1);
+          ldsm_x4_t(a0, a1, a2, a3, vs_t + swz<D>(row, ch));
+          mma_bf16(o[i], a0, a1, a2, a3, bhi[0], bhi[1]);
+          mma_bf16(o[i], a0, a1, a2, a3, blo[0], blo[1]);
+        }
       }
     }
     cp_async_wait<0>();
@@ -336,12 +327,16 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
       l += __shfl_xor_sync(0xffffffffu, l, 16);
       const int m = 8 * wig + 2 * cq + e;
       if (m >= p.M) continue;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l > 0.f ? vsref / l : 0.f;
       float *orow = direct ? p.o_part + out_row(p, s_idx, r, g, m) * D : p.ws_o + (wslot * p.M + m) * D;
+      if constexpr (FP8) {
+        store_col_fp8<D>(orow, [&](int i, int k) { return o[i][k]; }, e, gq, inv);
+      } else {
 #pragma unroll
-      for (int i = 0; i < MD; ++i) {
-        orow[16 * i + gq] = o[i][e] * inv;
-        orow[16 * i + gq + 8] = o[i][2 + e] * inv;
+        for (int i = 0; i < MD; ++i) {
+          orow[16 * i + gq] = o[i][e] * inv;
+          orow[16 * i + gq + 8] = o[i][2 + e] * inv;
+        }
       }
       if (gq == 0) {
         const float lse = l > 0.f ? (mcol[e] + __log2f(l)) * kLn2 : -INFINITY;
