@@ -370,8 +370,14 @@ __device__ __forceinline__ int swz(int row, int ch) {
 }
 
 // ------------------------------------------------------- fp32 K/V path --
-// Plain CUDA-core path for fp32 caches: warp w handles rows w, w+4, ...,
-// online softmax over the chunk's tokens read straight from global memory.
+// Plain CUDA-core path for fp32 caches.  The CTA stages the chunk's K and V
+// rows 32 tokens at a time in shared memory; warp w holds query rows w,
+// w + 4, ... .  For each tile a lane scores one token against the warp's
+// rows (dot products from shared memory, no shuffles), the online softmax
+// runs across the warp (one max and one sum per row and tile), and a lane
+// accumulates D / 32 output dims over the tile's tokens.
+constexpr int kF32Tile = 32;
+
 template <int D>
 struct F32Smem {
   TokMeta tm;
@@ -379,6 +385,10 @@ struct F32Smem {
   float o[kMaxRows * D];
   float lse[kMaxRows];
   float scratch[kMaxRows * (4096 / kMinChunkBlocks + 2 + kMaxSplits)];  // nch * M floats
+  alignas(16) float q[kMaxRows][D];
+  alignas(16) float kt[kF32Tile][D + 4];  // padded rows: the per-lane row reads miss no bank
+  alignas(16) float vt[kF32Tile][D];
+  float pt[kWarps][kMaxRows / kWarps][kF32Tile];
   int flag;
 };
 
@@ -396,39 +406,101 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_f32_kernel(Params p) {
   if (chunk == 0) write_empty_splits<D>(p, pl, r, g);
   if (!pl.active) return;
   fill_meta<D>(p, pl, r, g, sm.tm);
-  __syncthreads();
   constexpr int kPer = D / 32;
+  constexpr int kR = kMaxRows / kWarps;  // rows per warp
   const float *kc = static_cast<const float *>(p.c.k_cache);
   const float *vc = static_cast<const float *>(p.c.v_cache);
-  const float *q = static_cast<const float *>(p.q);
+  const float *qg = static_cast<const float *>(p.q);
+  for (int i = tid; i < p.M * D; i += kThreads) {
+    const int m = i / D, d = i % D;
+    sm.q[m][d] = qg[(((long long)r * p.T + m / p.G) * p.Hq + g * p.G + m % p.G) * D + d];
+  }
   const int ntok = (pl.e_end - pl.e_begin) * 4;
-  for (int m = warp; m < p.M; m += kWarps) {
-    const int t = m / p.G, h = g * p.G + m % p.G;
-    const int pt = pl.p0 + t;
-    float qv[kPer], acc[kPer];
-    for (int j = 0; j < kPer; ++j) {
-      qv[j] = q[(((long long)r * p.T + t) * p.Hq + h) * D + lane + 32 * j];
-      acc[j] = 0.f;
-    }
-    float mx = -INFINITY, l = 0.f;
-    for (int k = 0; k < ntok; ++k) {
-      const int pos = sm.tm.pos[k];
-      if (!(pos >= 0 && pos <= pt && (sm.tm.insel[k] || pos > pl.p0))) continue;
-      const long long off = sm.tm.off[k];
-      float d = 0.f;
-      for (int j = 0; j < kPer; ++j) d += qv[j] * kc[off + lane + 32 * j];
+  const int p0 = pl.p0;
+  float acc[kR][kPer], mx[kR], l[kR];
+  int tq[kR];  // query token of each row, -1: no row
 #pragma unroll
-      for (int o2 = 16; o2 >= 1; o2 >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o2);
-      const float x = d * p.scale_log2;
-      const float mn = fmaxf(mx, x);
-      const float a = exp2f(mx - mn);
-      const float w = exp2f(x - mn);
-      l = l * a + w;
-      for (int j = 0; j < kPer; ++j) acc[j] = acc[j] * a + w * vc[off + lane + 32 * j];
-      mx = mn;
+  for (int i = 0; i < kR; ++i) {
+    const int m = warp + kWarps * i;
+    tq[i] = m < p.M ? m / p.G : -1;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) acc[i][j] = 0.f;
+    mx[i] = -INFINITY;
+    l[i] = 0.f;
+  }
+  for (int k0 = 0; k0 < ntok; k0 += kF32Tile) {
+    __syncthreads();  // metadata and q written; the previous tile consumed
+    for (int i = tid; i < kF32Tile * D / 4; i += kThreads) {
+      const int t = i / (D / 4), d = 4 * (i % (D / 4));
+      const long long off = sm.tm.off[k0 + t];  // -1: no token (slots past the chunk too)
+      float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
+      if (off >= 0) {
+        kv = *reinterpret_cast<const float4 *>(kc + off + d);
+        vv = *reinterpret_cast<const float4 *>(vc + off + d);
+      }
+      *reinterpret_cast<float4 *>(&sm.kt[t][d]) = kv;
+      *reinterpret_cast<float4 *>(&sm.vt[t][d]) = vv;
     }
-    for (int j = 0; j < kPer; ++j) sm.o[m * D + lane + 32 * j] = l > 0.f ? acc[j] / l : 0.f;
-    if (lane == 0) sm.lse[m] = l > 0.f ? (mx + __log2f(l)) * kLn2 : -INFINITY;
+    __syncthreads();
+    // scores of token k0 + lane against the warp's rows
+    float sc[kR];
+#pragma unroll
+    for (int i = 0; i < kR; ++i) sc[i] = 0.f;
+#pragma unroll 4
+    for (int d = 0; d < D; d += 4) {
+      const float4 kv = *reinterpret_cast<const float4 *>(&sm.kt[lane][d]);
+#pragma unroll
+      for (int i = 0; i < kR; ++i) {
+        if (tq[i] < 0) continue;
+        const float4 qv = *reinterpret_cast<const float4 *>(&sm.q[warp + kWarps * i][d]);
+        sc[i] += kv.x * qv.x + kv.y * qv.y + kv.z * qv.z + kv.w * qv.w;
+      }
+    }
+    const int pos = sm.tm.pos[k0 + lane];
+    const bool ins = sm.tm.insel[k0 + lane];
+#pragma unroll
+    for (int i = 0; i < kR; ++i) {
+      if (tq[i] < 0) continue;
+      const bool vis = pos >= 0 && pos <= p0 + tq[i] && (ins || pos > p0);
+      const float x = vis ? sc[i] * p.scale_log2 : -INFINITY;
+      float mt = x;
+#pragma unroll
+      for (int o2 = 16; o2 >= 1; o2 >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o2));
+      const float mn = fmaxf(mx[i], mt);
+      const float base = (mn == -INFINITY) ? 0.f : mn;
+      const float a = (mn == -INFINITY) ? 1.f : exp2f(mx[i] - base);
+      const float pv = exp2f(x - base);  // 0 for an invisible token
+      float ps = pv;
+#pragma unroll
+      for (int o2 = 16; o2 >= 1; o2 >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o2);
+      l[i] = l[i] * a + ps;
+      mx[i] = mn;
+      sm.pt[warp][i][lane] = pv;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) acc[i][j] *= a;
+    }
+    __syncwarp();
+#pragma unroll 4
+    for (int t = 0; t < kF32Tile; ++t) {
+      float vv[kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) vv[j] = sm.vt[t][lane + 32 * j];
+#pragma unroll
+      for (int i = 0; i < kR; ++i) {
+        if (tq[i] < 0) continue;
+        const float pw = sm.pt[warp][i][t];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) acc[i][j] += pw * vv[j];
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kR; ++i) {
+    const int m = warp + kWarps * i;
+    if (m >= p.M) continue;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) sm.o[m * D + lane + 32 * j] = l[i] > 0.f ? acc[i][j] / l[i] : 0.f;
+    if (lane == 0) sm.lse[m] = l[i] > 0.f ? (mx[i] + __log2f(l[i])) * kLn2 : -INFINITY;
   }
   __syncthreads();
   finish_chunk<D>(p, pl, r, g, sm.o, sm.lse, &sm.flag, sm.scratch);
