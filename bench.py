@@ -40,6 +40,9 @@ def parse_args(argv=None):
     ap.add_argument("--splits", type=int, default=2)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (profiling runs only)")
+    ap.add_argument("--ctx", default=None,
+                    help="override the workload's context lengths, e.g. fixed:16384 "
+                         "(profiling runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--dcp", action="store_true",
@@ -330,9 +333,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = WORKLOADS[args.workload]
-    if args.batch is not None:
+    if args.batch is not None or args.ctx is not None:
         from dataclasses import replace
-        w = replace(w, batch=args.batch)
+        w = replace(w, batch=args.batch if args.batch is not None else w.batch,
+                    ctx=args.ctx if args.ctx is not None else w.ctx)
     dcp = args.dcp and world > 1
     S = world if dcp else args.splits
     # replicas draw independent batches; DCP ranks share one batch
