@@ -88,7 +88,8 @@ def weak_scaling_rate(per_rank_units: int, world: int, steps: int, ms_max: float
 def algorithmic_bytes(w, L: int, num_splits: int) -> dict:
     """Bytes one query (one request, T query tokens) must move.
 
-    index_topk : every competing compressed key (int16, d per block), the
+    index_topk : every competing compressed key (packed: d low bytes and d/4
+                 bytes of 2-bit high fields per block), the
                  block-table entries of those pages, the indexer query and
                  the selection row written.
     sparse_decode : K and V rows of the selected tokens for every kv head,
@@ -104,13 +105,14 @@ def algorithmic_bytes(w, L: int, num_splits: int) -> dict:
     pages = math.ceil(n * 4 / P)
     topk = min(w.topk, n)
     tokens = topk * 4 + (w.T - 1)
-    idx = n * w.d_idx * 2 + pages * 4 + w.d_idx + w.topk * 4
+    kc_block = w.d_idx + w.d_idx // 4
+    idx = n * kc_block + pages * 4 + w.d_idx + w.topk * 4
     dec = (2 * tokens * w.Hkv * w.D * kv_elem + w.T * w.Hq * w.D * q_elem + w.topk * 4
            + num_splits * w.T * w.Hq * (w.D + 1) * 4)
     if w.kv_dtype == "e4m3":
         dec += 2 * min(tokens, math.ceil(L / P)) * w.Hkv * 4
     merge = num_splits * w.T * w.Hq * (w.D + 1) * 4 + w.T * w.Hq * (w.D + 1) * 4
-    append = w.T * w.d_idx * 3 + 2 * w.d_idx * 2
+    append = w.T * w.d_idx * 3 + 2 * kc_block
     return dict(index_topk=idx, sparse_decode=dec, lse_merge=merge, compress_append=append,
                 total=idx + dec + merge + append)
 

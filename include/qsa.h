@@ -73,7 +73,9 @@ typedef struct {
   const void *v_cache;  /* [num_pages, P, Hkv, D] of kv_dtype                 */
   const float *k_scale; /* [num_pages, Hkv] dequant scale (FP8 only, else NULL) */
   const float *v_scale; /* [num_pages, Hkv] dequant scale (FP8 only, else NULL) */
-  int16_t *kc;          /* [num_pages, P/4, d] compressed keys (sum of 4 int8 keys) */
+  uint8_t *kc;          /* [num_pages, qsa_kc_page_bytes(P, d)] packed compressed
+                           keys (sums of 4 int8 keys), 16-byte aligned; layout
+                           at qsa_kc_page_bytes                               */
   int8_t *ring;         /* [ring_rows, 4, d] raw keys of the newest positions:
                            slot p % 4 of row r holds request r's key at p     */
   int32_t ring_rows;    /* rows of `ring` (>= batch of every call)            */
@@ -87,6 +89,25 @@ const char *qsa_status_string(int32_t status);
 
 /* Library ABI version (incremented on any incompatible change). */
 int32_t qsa_abi_version(void);
+
+/*
+ * qsa_kc_page_bytes — bytes of one page of the packed compressed-key cache,
+ * or 0 for an unsupported geometry (page_size not a positive multiple of 4,
+ * idx_dim not 32, 64 or 128).
+ *
+ * A compressed key value v of micro-block b, dim j (the sum of 4 int8 keys,
+ * -512 <= v <= 508) is stored losslessly in 10 bits: its low byte v & 255
+ * and a 2-bit high field f = (v >> 8) + 2 in [0, 3], so v = 256 (f - 2) +
+ * low byte.  A page of P tokens (R = P/4 micro-blocks, d = idx_dim) holds
+ *   bytes [0, R*d)             R rows of d low bytes (row = micro-block in
+ *                              the page, column = dim),
+ *   bytes [R*d, R*d + R*d/4)   R rows of d/4 high-field bytes,
+ * then zero padding to a multiple of 16 bytes.  In a high row, dims 16w ..
+ * 16w+15 form the little-endian 32-bit word w, dim 16w + 4s + k (s, k in
+ * [0, 4)) at bits 8k + 2s.  (The int16 layout would move 2d bytes per
+ * micro-block through the scan of qsa_index_topk; this one 1.25 d.)
+ */
+size_t qsa_kc_page_bytes(int32_t page_size, int32_t idx_dim);
 
 /*
  * qsa_compress_append — write new tokens' raw indexer keys and refresh the

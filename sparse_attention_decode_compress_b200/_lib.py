@@ -28,6 +28,7 @@ class QsaCacheStruct(ctypes.Structure):
 SIGNATURES = {
     "qsa_status_string": (ctypes.c_char_p, [c_int32]),
     "qsa_abi_version": (c_int32, []),
+    "qsa_kc_page_bytes": (c_size_t, [c_int32, c_int32]),
     "qsa_compress_append": (c_int32, [ctypes.POINTER(QsaCacheStruct), c_int32, c_void_p, c_void_p,
                                       c_void_p, c_int32, c_void_p]),
     "qsa_index_topk_workspace_bytes": (c_size_t, [c_int32, c_int32]),

@@ -58,7 +58,7 @@ class QSACache:
     compressed-key cache)."""
     k_cache: torch.Tensor               # [num_pages, P, Hkv, D] f32 / bf16 / fp8 e4m3
     v_cache: torch.Tensor
-    kc: torch.Tensor                    # int16 [num_pages, P/4, d]
+    kc: torch.Tensor                    # uint8 [num_pages, qsa_kc_page_bytes(P, d)], packed
     ring: torch.Tensor                  # int8 [ring_rows, 4, d]
     block_table: torch.Tensor           # int32 [B, max_pages]
     k_scale: torch.Tensor | None = None  # f32 [num_pages, Hkv] (fp8 only)
@@ -68,7 +68,10 @@ class QSACache:
     def allocate(k_cache, v_cache, block_table, idx_dim: int, ring_rows: int,
                  k_scale=None, v_scale=None) -> "QSACache":
         num_pages, P = k_cache.shape[0], k_cache.shape[1]
-        kc = torch.zeros((num_pages, P // 4, idx_dim), dtype=torch.int16, device=k_cache.device)
+        page_bytes = int(_lib.load().qsa_kc_page_bytes(P, idx_dim))
+        if page_bytes == 0:
+            raise ValueError(f"unsupported compressed-key geometry: page_size {P}, idx_dim {idx_dim}")
+        kc = torch.zeros((num_pages, page_bytes), dtype=torch.uint8, device=k_cache.device)
         ring = torch.zeros((ring_rows, 4, idx_dim), dtype=torch.int8, device=k_cache.device)
         return QSACache(k_cache, v_cache, kc, ring, block_table, k_scale, v_scale)
 
@@ -77,13 +80,15 @@ class QSACache:
         if k.dtype not in _KV_DTYPES or v.dtype != k.dtype or k.shape != v.shape or k.dim() != 4:
             raise TypeError("k_cache / v_cache must be [num_pages, P, Hkv, D] of one dtype "
                             "(float32, bfloat16 or float8_e4m3fn)")
-        _need(self.kc, torch.int16, "kc")
+        _need(self.kc, torch.uint8, "kc")
         _need(self.ring, torch.int8, "ring")
         _need(self.block_table, torch.int32, "block_table")
         num_pages, P, Hkv, D = k.shape
-        d = self.kc.shape[-1]
-        if self.kc.shape != (num_pages, P // 4, d) or self.ring.shape[1:] != (4, d):
-            raise ValueError("kc must be [num_pages, P/4, d] and ring [rows, 4, d]")
+        d = self.ring.shape[-1]
+        page_bytes = int(_lib.load().qsa_kc_page_bytes(P, d))
+        if self.ring.dim() != 3 or self.ring.shape[1] != 4 or page_bytes == 0 or \
+                self.kc.shape != (num_pages, page_bytes):
+            raise ValueError("ring must be [rows, 4, d] and kc [num_pages, qsa_kc_page_bytes(P, d)]")
         s = _lib.QsaCacheStruct()
         s.num_pages, s.page_size, s.num_kv_heads, s.head_dim, s.idx_dim = num_pages, P, Hkv, D, d
         s.kv_dtype = _KV_DTYPES[k.dtype]
@@ -308,7 +313,7 @@ class QSASession:
         self._struct = cache.struct()
         self.B, self.T, self.Hq, self.topk = B, T, Hq, topk
         self.D = cache.k_cache.shape[-1]
-        self.d = cache.kc.shape[-1]
+        self.d = cache.ring.shape[-1]
         self.q_dtype = q_dtype
         qd = {torch.float32: _lib.QSA_F32, torch.bfloat16: _lib.QSA_BF16}[q_dtype]
         lib = _lib.load()

@@ -7,11 +7,12 @@
 // padded with -1).  score = exact int32 dot(q_idx, kc); ties -> lower block
 // index; kept blocks listed in ascending order.
 //
-// Design (B200): the scan is an HBM stream of int16 compressed keys
-// (256 B per block at d = 128).  Persistent warps walk 8 KiB items (request,
-// run of rows), load them with 16-byte streaming loads (16 per lane in
-// flight), turn them into scores with dp2a (int16 x int8 pairs) and a
-// butterfly reduce-scatter, and write the scores to an L2-resident buffer.
+// Design (B200): the scan is an HBM stream of packed compressed keys (160 B
+// per block at d = 128: a low byte and a 2-bit high field per dim, see
+// qsa_common.cuh).  Persistent warps walk items of 64 rows (request, run of
+// rows), load them with streaming loads (16 + 4 bytes per lane and row, 16
+// rows per lane in flight), turn them into scores with dp4a and a butterfly
+// reduce-scatter, and write the scores to an L2-resident buffer.
 // A second kernel selects, one CTA per request: a 4096-bin histogram of the
 // high score bits finds the threshold bin, the blocks above it are kept
 // outright, the threshold bin's blocks are gathered in shared memory and
@@ -536,7 +537,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
 // are fetched while the current one computes.
 
 constexpr int kScanThreads = 128;
-constexpr int kItemLoads = 16;  // 16-byte loads per lane per item (8 KiB per warp)
+constexpr int kItemLoads = 16;  // 16-byte key loads per lane per item (8 KiB of low bytes per warp)
 
 __device__ __forceinline__ int pow2_log(int x) { return 31 - __clz(x); }
 
@@ -591,7 +592,7 @@ struct ItemWalker {
 };
 
 #ifndef QSA_SCAN_MIN_CTAS
-#define QSA_SCAN_MIN_CTAS 5
+#define QSA_SCAN_MIN_CTAS 4
 #endif
 #ifndef QSA_SCAN_LOAD
 #define QSA_SCAN_LOAD 2
@@ -631,21 +632,47 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   return pol;
 }
 
+// 4-byte load of high key fields, read once per call (L1 bypassed, L2
+// evict-first).
+__device__ __forceinline__ uint32_t scan_load32(const uint32_t *p, uint64_t policy) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.b32 %0, [%1], %2;"
+               : "=r"(v) : "l"(p), "l"(policy));
+  return v;
+}
+// Dot product of four unsigned bytes (a) with four signed bytes (b), plus c.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // BPPC: micro-blocks per page when it is a compile-time constant (16 for
 // 64-token pages, 4 for 16-token pages), 0 for any page size.
+//
+// Keys are the packed pages of qsa_common.cuh.  A lane owns 16 dims of a row:
+// one 16-byte load of low bytes and one 4-byte load of high fields.  With
+// v = 256 (f - 2) + lo, the score is
+//   sum q*lo + 256 * sum q*f - 512 * sum q,
+// the first two by dp4a (unsigned key bytes, signed query bytes), the last a
+// constant of the request.
 template <int DI, int BPPC>
 __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_kernel(Params p) {
   pdl_open();
-  constexpr int kLPR = DI / 8;                    // lanes per row (16 B each)
+  static_assert(DI == 32 || DI == 64 || DI == 128, "indexer dim");
+  constexpr int kLPR = DI / 16;                   // lanes per row (16 dims each)
   constexpr int kRPI = 32 / kLPR;                 // rows per load instruction
-  constexpr int kRowsPerItem = kItemLoads * kRPI; // 4096 / DI
-  constexpr int kR = (kLPR == 16) ? 4 : (kLPR == 8) ? 3 : 2;
+  constexpr int kRowsPerItem = kItemLoads * kRPI; // 8192 / DI
+  constexpr int kR = (kLPR == 8) ? 3 : (kLPR == 4) ? 2 : 1;  // log2(kLPR)
   constexpr int kVals = 16 >> kR;
+  constexpr int kHiRow = DI / 4;                  // high-field bytes per row
   const int lane = threadIdx.x & 31;
   const long long warp_id = ((long long)blockIdx.x * kScanThreads + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * kScanThreads) >> 5;
   const int bpp = p.c.page_size / 4;
-  const int sub = lane % kLPR;                    // this lane's 8 dims: 8*sub .. 8*sub+7
+  const long long page_bytes = kc_page_bytes(p.c.page_size, DI);
+  const long long lo_bytes = kc_lo_bytes(p.c.page_size, DI);
+  const int sub = lane % kLPR;                    // this lane's dims: 16*sub .. 16*sub+15
   const int row_in = lane / kLPR;
 
   const uint64_t pol_stream = l2_policy_evict_first();
@@ -653,7 +680,8 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
   ItemWalker wk;
   wk.start(p, kRowsPerItem, warp_id == 0 && lane == 0);
   int cur_r = -1;
-  uint32_t q0 = 0, q1 = 0;
+  uint32_t q[4] = {0u, 0u, 0u, 0u};
+  int qbias = 0;
 
   // block-table entries of an item: lane j holds logical page lp0 + j
   // (rows and logical pages fit in 32 bits: n <= max_blocks <= 2^24)
@@ -683,11 +711,18 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
     const int n = wk.n;
     if (r != cur_r) {
       cur_r = r;
-      const uint2 qq = *reinterpret_cast<const uint2 *>(p.q_idx + (long long)r * DI + sub * 8);
-      q0 = qq.x;
-      q1 = qq.y;
+      const uint32_t *qw = reinterpret_cast<const uint32_t *>(p.q_idx + (long long)r * DI + sub * 16);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) q[j] = qw[j];
+      int qs = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) qs = dp4a_us(0x01010101u, q[j], qs);
+#pragma unroll
+      for (int o = 1; o < kLPR; o <<= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+      qbias = -512 * qs;
     }
     uint4 v[kItemLoads];
+    uint32_t h[kItemLoads];
     constexpr int kB = BPPC > 0 ? BPPC : 1;  // keeps the constant arithmetic defined
     constexpr bool kFixed = BPPC > 0 && (kB % kRPI == 0) &&
                             (kRowsPerItem % kB == 0 || kB % kRowsPerItem == 0);
@@ -696,24 +731,26 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
       // one page base per page of the item, constant offsets per load; an
       // invalid page reads page 0 instead (scores garbage, error recorded)
       constexpr int kPagesPerItem = kRowsPerItem >= kB ? kRowsPerItem / kB : 1;
-      const int16_t *base[kPagesPerItem];
+      const uint8_t *base[kPagesPerItem];
 #pragma unroll
-      for (int q = 0; q < kPagesPerItem; ++q) {
-        const int j = (row0 + q * kB) / kB - lp0;  // 0 .. kPagesPerItem-1 here
+      for (int qq = 0; qq < kPagesPerItem; ++qq) {
+        const int j = (row0 + qq * kB) / kB - lp0;  // 0 .. kPagesPerItem-1 here
         int pg = __shfl_sync(0xffffffffu, pg_lane, j & 31);
         if (pg < 0) {
           if (lane == 0) record_error(kErrBounds);
           pg = 0;
         }
-        base[q] = p.c.kc + ((long long)pg * kB + (kRowsPerItem >= kB ? 0 : row0 % kB)) * DI;
+        base[qq] = p.c.kc + (long long)pg * page_bytes;
       }
+      const int rp0 = kRowsPerItem >= kB ? 0 : row0 % kB;  // first row of the item in its page
 #pragma unroll
       for (int i = 0; i < kItemLoads; ++i) {
         const int rr = i * kRPI;  // row of load i (before row_in) within the item
-        const int q = kRowsPerItem >= kB ? rr / kB : 0;
-        const int rin = kRowsPerItem >= kB ? rr % kB : rr;
-        v[i] = scan_load(reinterpret_cast<const uint4 *>(base[q] + (rin + row_in) * DI + sub * 8),
-                         pol_stream);
+        const int qq = kRowsPerItem >= kB ? rr / kB : 0;
+        const int rin = rp0 + (kRowsPerItem >= kB ? rr % kB : rr) + row_in;
+        v[i] = scan_load(reinterpret_cast<const uint4 *>(base[qq] + rin * DI + sub * 16), pol_stream);
+        h[i] = scan_load32(
+            reinterpret_cast<const uint32_t *>(base[qq] + lo_bytes + rin * kHiRow + sub * 4), pol_stream);
       }
     } else {
     // issue this item's loads; the lane's row advances by kRPI per load, so
@@ -730,11 +767,14 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
         if (pg >= p.c.num_pages) pg = -1;
       }
       v[i] = make_uint4(0, 0, 0, 0);
+      h[i] = 0u;
       if (row < n) {
         if (pg >= 0) {
-          const uint4 *src = reinterpret_cast<const uint4 *>(
-              p.c.kc + ((long long)pg * bpp + off) * DI + sub * 8);
-          v[i] = scan_load(src, pol_stream);
+          const uint8_t *pb = p.c.kc + (long long)pg * page_bytes;
+          v[i] = scan_load(reinterpret_cast<const uint4 *>(pb + (long long)off * DI + sub * 16), pol_stream);
+          h[i] = scan_load32(
+              reinterpret_cast<const uint32_t *>(pb + lo_bytes + (long long)off * kHiRow + sub * 4),
+              pol_stream);
         } else if (lane == 0 || sub == 0) {
           record_error(kErrBounds);
         }
@@ -754,14 +794,19 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
       nrow0 = (int)(it - wk.cum) * kRowsPerItem;
       npg = fetch_pages(nr, nrow0, nlp0);
     }
-    // scores: dp2a of int16 pairs with int8 query pairs
+    // partial scores of the lane's 16 dims: low bytes and high fields
     int acc[16];
 #pragma unroll
     for (int i = 0; i < kItemLoads; ++i) {
-      int a = __dp2a_lo((int)v[i].x, (int)q0, 0);
-      a = __dp2a_hi((int)v[i].y, (int)q0, a);
-      a = __dp2a_lo((int)v[i].z, (int)q1, a);
-      acc[i] = __dp2a_hi((int)v[i].w, (int)q1, a);
+      int a = dp4a_us(v[i].x, q[0], 0);
+      a = dp4a_us(v[i].y, q[1], a);
+      a = dp4a_us(v[i].z, q[2], a);
+      a = dp4a_us(v[i].w, q[3], a);
+      int b = dp4a_us(h[i] & 0x03030303u, q[0], 0);
+      b = dp4a_us((h[i] >> 2) & 0x03030303u, q[1], b);
+      b = dp4a_us((h[i] >> 4) & 0x03030303u, q[2], b);
+      b = dp4a_us((h[i] >> 6) & 0x03030303u, q[3], b);
+      acc[i] = a + (b << 8);
     }
     reduce_scatter16<kLPR>(acc, lane);
     int32_t *sc = p.scores + (long long)r * p.max_blocks;
@@ -769,7 +814,7 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
     for (int k = 0; k < kVals; ++k) {
       const int i = ((lane % kLPR) << (4 - kR)) | k;
       const int row = row0 + i * kRPI + row_in;
-      if (row < n) score_store(sc + row, acc[k], pol_keep);
+      if (row < n) score_store(sc + row, acc[k] + qbias, pol_keep);
     }
     if (!more) break;
   }

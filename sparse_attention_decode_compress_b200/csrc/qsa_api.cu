@@ -320,7 +320,13 @@ const char *qsa_status_string(int32_t status) {
   }
 }
 
-int32_t qsa_abi_version(void) { return 1; }
+int32_t qsa_abi_version(void) { return 2; }
+
+size_t qsa_kc_page_bytes(int32_t page_size, int32_t idx_dim) {
+  if (page_size <= 0 || page_size % 4 != 0) return 0;
+  if (idx_dim != 32 && idx_dim != 64 && idx_dim != 128) return 0;
+  return (size_t)qsa::kc_page_bytes(page_size, idx_dim);
+}
 
 qsa_status qsa_compress_append(const qsa_cache *cache, int32_t B, const int32_t *pos0,
                                const int32_t *cu_new, const int8_t *k_new,
@@ -331,7 +337,7 @@ qsa_status qsa_compress_append(const qsa_cache *cache, int32_t B, const int32_t 
   if (B == 0 || max_new_per_req == 0) return QSA_OK;
   if (B > cache->ring_rows || B > 65535) return QSA_ERR_INVALID_ARG;
   if (!pos0 || !cu_new || !k_new || !cache->kc || !cache->ring) return QSA_ERR_INVALID_ARG;
-  if (!aligned(k_new, 4) || !aligned(cache->kc, 8) || !aligned(cache->ring, 4))
+  if (!aligned(k_new, 4) || !aligned(cache->kc, 16) || !aligned(cache->ring, 4))
     return QSA_ERR_INVALID_ARG;
   const long long max_blocks = (long long)max_new_per_req / 4 + 2;
   const long long gx = (max_blocks + qsa::kAppendBlocksPerCta - 1) / qsa::kAppendBlocksPerCta;

@@ -120,10 +120,25 @@ def oracle_request(batch: QSABatch, r: int, num_splits: int) -> dict:
     return out
 
 
+def unpack_kc_pages(pages: np.ndarray, P: int, d: int) -> np.ndarray:
+    """Compressed-key values [n, P/4, d] (int64) of packed pages [n, bytes],
+    read by the layout include/qsa.h states at qsa_kc_page_bytes: R = P/4
+    rows of d low bytes, then R rows of d/4 high-field bytes, dim 16w+4s+k
+    of a row at bits 8k+2s of its 32-bit word w; value = 256*(field-2)+low."""
+    R = P // 4
+    n = pages.shape[0]
+    lo = pages[:, :R * d].reshape(n, R, d).astype(np.int64)
+    hib = pages[:, R * d:R * d + R * d // 4].reshape(n, R, d // 16, 4).astype(np.int64)
+    s = np.arange(4)
+    f = (hib[:, :, :, None, :] >> (2 * s)[:, None]) & 3   # [n, R, w, s, k]
+    return 256 * (f.reshape(n, R, d) - 2) + lo
+
+
 def gpu_kc_logical(batch: QSABatch, cache: QSACache, r: int) -> np.ndarray:
     L = int(batch.ctx_lens_host[r])
     pages = request_pages(batch, r)
-    kcp = cache.kc[pages.to(batch.device)].cpu().numpy()
+    kcp = unpack_kc_pages(cache.kc[pages.to(batch.device)].cpu().numpy(), batch.w.page_size,
+                          batch.w.d_idx)
     return ref.depage_kc(kcp, np.arange(pages.shape[0]), L, batch.w.page_size)
 
 

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings_and_version():
     lib = _lib.load()
-    assert lib.qsa_abi_version() == 1
+    assert lib.qsa_abi_version() == 2
     assert lib.qsa_status_string(0) == b"QSA_OK"
     assert b"BOUNDS" in lib.qsa_status_string(3)
     assert b"unknown" in lib.qsa_status_string(99)

@@ -1,0 +1,49 @@
+"""The packed compressed-key page layout of include/qsa.h
+(qsa_kc_page_bytes): page sizes from the library, and the test harness's
+reader of the layout against pages packed here field by field."""
+import numpy as np
+import pytest
+
+import qsa_harness as H
+from sparse_attention_decode_compress_b200 import _lib
+
+
+def _pack(vals: np.ndarray, P: int, d: int, page_bytes: int) -> np.ndarray:
+    """Packs values [n, P/4, d] in [-512, 508] one field at a time."""
+    n, R, _ = vals.shape
+    out = np.zeros((n, page_bytes), dtype=np.uint8)
+    for pg in range(n):
+        for row in range(R):
+            for j in range(d):
+                v = int(vals[pg, row, j])
+                out[pg, row * d + j] = v & 255
+                f = (v >> 8) + 2
+                w, s, k = j // 16, (j % 16) // 4, j % 4
+                out[pg, R * d + row * (d // 4) + 4 * w + k] |= f << (2 * s)
+    return out
+
+
+@pytest.mark.parametrize("P,d", [(64, 128), (16, 32), (64, 64), (4, 32), (16, 128)])
+def test_page_bytes(P, d):
+    lib = _lib.load()
+    R = P // 4
+    assert lib.qsa_kc_page_bytes(P, d) == R * d + -(-(R * d // 4) // 16) * 16
+    assert lib.qsa_kc_page_bytes(P, d) % 16 == 0
+
+
+def test_page_bytes_rejects_bad_geometry():
+    lib = _lib.load()
+    assert lib.qsa_kc_page_bytes(6, 128) == 0
+    assert lib.qsa_kc_page_bytes(64, 48) == 0
+    assert lib.qsa_kc_page_bytes(0, 128) == 0
+
+
+@pytest.mark.parametrize("P,d", [(64, 128), (16, 32), (8, 64)])
+def test_harness_reader_round_trip(P, d):
+    lib = _lib.load()
+    rng = np.random.default_rng(P * d)
+    vals = rng.integers(-512, 509, size=(3, P // 4, d))
+    vals[0, 0, :4] = [-512, 508, -1, 0]   # extremes and the field boundary
+    vals[0, 0, 4:8] = [255, 256, -256, -257]
+    pages = _pack(vals, P, d, int(lib.qsa_kc_page_bytes(P, d)))
+    assert np.array_equal(H.unpack_kc_pages(pages, P, d), vals)
