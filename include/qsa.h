@@ -64,7 +64,8 @@ typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype;
  * block-table entry names the same physical page in all of them. */
 typedef struct {
   int32_t num_pages;    /* physical pages in each cache                       */
-  int32_t page_size;    /* tokens per page P; multiple of 4 (compress ratio)  */
+  int32_t page_size;    /* tokens per page P; multiple of 16 (4-token micro-
+                           blocks, packed compressed keys in runs of 4)      */
   int32_t num_kv_heads; /* Hkv                                                */
   int32_t head_dim;     /* D: 64 or 128                                       */
   int32_t idx_dim;      /* indexer dim d: 32, 64 or 128                       */
@@ -92,8 +93,9 @@ int32_t qsa_abi_version(void);
 
 /*
  * qsa_kc_page_bytes — bytes of one page of the packed compressed-key cache,
- * or 0 for an unsupported geometry (page_size not a positive multiple of 4,
- * idx_dim not 32, 64 or 128).
+ * or 0 for an unsupported geometry (page_size not a positive multiple of 16,
+ * idx_dim not 32, 64 or 128).  qsa_compress_append and qsa_index_topk return
+ * QSA_ERR_UNSUPPORTED for a page_size that is not a multiple of 16.
  *
  * A compressed key value v of micro-block b, dim j (the sum of 4 int8 keys,
  * -512 <= v <= 508) is stored losslessly in 10 bits: its low byte v & 255
@@ -101,11 +103,13 @@ int32_t qsa_abi_version(void);
  * low byte.  A page of P tokens (R = P/4 micro-blocks, d = idx_dim) holds
  *   bytes [0, R*d)             R rows of d low bytes (row = micro-block in
  *                              the page, column = dim),
- *   bytes [R*d, R*d + R*d/4)   R rows of d/4 high-field bytes,
- * then zero padding to a multiple of 16 bytes.  In a high row, dims 16w ..
- * 16w+15 form the little-endian 32-bit word w, dim 16w + 4s + k (s, k in
- * [0, 4)) at bits 8k + 2s.  (The int16 layout would move 2d bytes per
- * micro-block through the scan of qsa_index_topk; this one 1.25 d.)
+ *   bytes [R*d, R*d + R*d/4)   d/16 * R little-endian 32-bit words of high
+ *                              fields: word w*R + row holds dims 16w ..
+ *                              16w+15 of that row, dim 16w + 4s + k (s, k
+ *                              in [0, 4)) at bits 8k + 2s,
+ * then zero padding to a multiple of 16 bytes.  (The int16 layout would move
+ * 2d bytes per micro-block through the scan of qsa_index_topk; this one
+ * 1.25 d.)
  */
 size_t qsa_kc_page_bytes(int32_t page_size, int32_t idx_dim);
 
@@ -132,7 +136,8 @@ size_t qsa_kc_page_bytes(int32_t page_size, int32_t idx_dim);
  * are read back from ring row r).  A decode step passes T new tokens per
  * request; a prefill passes whole chunks (complete blocks are pooled
  * straight from k_new).  Errors: QSA_ERR_INVALID_ARG for null pointers,
- * B < 0, B > ring_rows, page_size % 4 != 0 or an unsupported idx_dim.
+ * B < 0, B > ring_rows or page_size % 4 != 0; QSA_ERR_UNSUPPORTED for
+ * page_size % 16 != 0 or an unsupported idx_dim.
  */
 qsa_status qsa_compress_append(const qsa_cache *cache, int32_t B, const int32_t *pos0,
                                const int32_t *cu_new, const int8_t *k_new,

@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kAppendThreads) compress_append_kernel(
     uint8_t *pg = c.kc + (long long)page * page_bytes;
     const int row = (int)(b % bpp);
     *reinterpret_cast<uint4 *>(pg + (long long)row * DI + 16 * dw) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    *reinterpret_cast<uint32_t *>(pg + lo_bytes + (long long)row * (DI / 4) + 4 * dw) = hi;
+    *reinterpret_cast<uint32_t *>(pg + lo_bytes + 4 * ((long long)dw * bpp + row)) = hi;
   }
 
   if (blockIdx.x != 0) return;

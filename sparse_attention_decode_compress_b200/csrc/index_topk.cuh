@@ -10,8 +10,8 @@
 // Design (B200): the scan is an HBM stream of packed compressed keys (160 B
 // per block at d = 128: a low byte and a 2-bit high field per dim, see
 // qsa_common.cuh).  Persistent warps walk items of 64 rows (request, run of
-// rows), load them with streaming loads (16 + 4 bytes per lane and row, 16
-// rows per lane in flight), turn them into scores with dp4a and a butterfly
+// rows), load them with 16-byte streaming loads (a lane's 16 rows in runs of
+// 4, 20 loads in flight), turn them into scores with dp4a and a butterfly
 // reduce-scatter, and write the scores to an L2-resident buffer.
 // A second kernel selects, one CTA per request: a 4096-bin histogram of the
 // high score bits finds the threshold bin, the blocks above it are kept
@@ -632,14 +632,6 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   return pol;
 }
 
-// 4-byte load of high key fields, read once per call (L1 bypassed, L2
-// evict-first).
-__device__ __forceinline__ uint32_t scan_load32(const uint32_t *p, uint64_t policy) {
-  uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.b32 %0, [%1], %2;"
-               : "=r"(v) : "l"(p), "l"(policy));
-  return v;
-}
 // Dot product of four unsigned bytes (a) with four signed bytes (b), plus c.
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
   int d;
@@ -650,9 +642,11 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
 // BPPC: micro-blocks per page when it is a compile-time constant (16 for
 // 64-token pages, 4 for 16-token pages), 0 for any page size.
 //
-// Keys are the packed pages of qsa_common.cuh.  A lane owns 16 dims of a row:
-// one 16-byte load of low bytes and one 4-byte load of high fields.  With
-// v = 256 (f - 2) + lo, the score is
+// Keys are the packed pages of qsa_common.cuh.  A lane owns 16 dims of its
+// rows, which come in runs of 4 consecutive rows: per run, four 16-byte
+// loads of low bytes and one 16-byte load of the run's four high-field words
+// (stored dim-group major, so they are contiguous).  With v = 256 (f - 2) +
+// lo, the score is
 //   sum q*lo + 256 * sum q*f - 512 * sum q,
 // the first two by dp4a (unsigned key bytes, signed query bytes), the last a
 // constant of the request.
@@ -661,19 +655,21 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
   pdl_open();
   static_assert(DI == 32 || DI == 64 || DI == 128, "indexer dim");
   constexpr int kLPR = DI / 16;                   // lanes per row (16 dims each)
-  constexpr int kRPI = 32 / kLPR;                 // rows per load instruction
+  constexpr int kRPI = 32 / kLPR;                 // lane groups = rows per load instruction
   constexpr int kRowsPerItem = kItemLoads * kRPI; // 8192 / DI
+  constexpr int kRun = 4;                         // consecutive rows of a lane
+  constexpr int kRuns = kItemLoads / kRun;
+  constexpr int kRunStride = kRun * kRPI;         // rows from one run of a lane to its next
   constexpr int kR = (kLPR == 8) ? 3 : (kLPR == 4) ? 2 : 1;  // log2(kLPR)
   constexpr int kVals = 16 >> kR;
-  constexpr int kHiRow = DI / 4;                  // high-field bytes per row
   const int lane = threadIdx.x & 31;
   const long long warp_id = ((long long)blockIdx.x * kScanThreads + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * kScanThreads) >> 5;
-  const int bpp = p.c.page_size / 4;
+  const int bpp = BPPC > 0 ? BPPC : p.c.page_size / 4;  // rows per page
   const long long page_bytes = kc_page_bytes(p.c.page_size, DI);
   const long long lo_bytes = kc_lo_bytes(p.c.page_size, DI);
   const int sub = lane % kLPR;                    // this lane's dims: 16*sub .. 16*sub+15
-  const int row_in = lane / kLPR;
+  const int grp = lane / kLPR;                    // this lane's runs start at row kRun*grp
 
   const uint64_t pol_stream = l2_policy_evict_first();
   const uint64_t pol_keep = l2_policy_evict_last();
@@ -721,70 +717,40 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
       for (int o = 1; o < kLPR; o <<= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
       qbias = -512 * qs;
     }
+    // issue the item's loads: run u of this lane is rows fr .. fr+3 of one
+    // page (runs are 4-aligned and a page holds a multiple of 4 rows); an
+    // invalid page is skipped (scores garbage, error recorded)
     uint4 v[kItemLoads];
-    uint32_t h[kItemLoads];
-    constexpr int kB = BPPC > 0 ? BPPC : 1;  // keeps the constant arithmetic defined
-    constexpr bool kFixed = BPPC > 0 && (kB % kRPI == 0) &&
-                            (kRowsPerItem % kB == 0 || kB % kRowsPerItem == 0);
-    if (kFixed && row0 + kRowsPerItem <= n) {
-      // whole item inside the request, page geometry known at compile time:
-      // one page base per page of the item, constant offsets per load; an
-      // invalid page reads page 0 instead (scores garbage, error recorded)
-      constexpr int kPagesPerItem = kRowsPerItem >= kB ? kRowsPerItem / kB : 1;
-      const uint8_t *base[kPagesPerItem];
+    uint4 hv[kRuns];
 #pragma unroll
-      for (int qq = 0; qq < kPagesPerItem; ++qq) {
-        const int j = (row0 + qq * kB) / kB - lp0;  // 0 .. kPagesPerItem-1 here
-        int pg = __shfl_sync(0xffffffffu, pg_lane, j & 31);
-        if (pg < 0) {
-          if (lane == 0) record_error(kErrBounds);
-          pg = 0;
-        }
-        base[qq] = p.c.kc + (long long)pg * page_bytes;
-      }
-      const int rp0 = kRowsPerItem >= kB ? 0 : row0 % kB;  // first row of the item in its page
-#pragma unroll
-      for (int i = 0; i < kItemLoads; ++i) {
-        const int rr = i * kRPI;  // row of load i (before row_in) within the item
-        const int qq = kRowsPerItem >= kB ? rr / kB : 0;
-        const int rin = rp0 + (kRowsPerItem >= kB ? rr % kB : rr) + row_in;
-        v[i] = scan_load(reinterpret_cast<const uint4 *>(base[qq] + rin * DI + sub * 16), pol_stream);
-        h[i] = scan_load32(
-            reinterpret_cast<const uint32_t *>(base[qq] + lo_bytes + rin * kHiRow + sub * 4), pol_stream);
-      }
-    } else {
-    // issue this item's loads; the lane's row advances by kRPI per load, so
-    // its (logical page, row in page) pair is stepped instead of divided
-    int lp = (row0 + row_in) / bpp;
-    int off = (row0 + row_in) - lp * bpp;
-#pragma unroll
-    for (int i = 0; i < kItemLoads; ++i) {
-      const int row = row0 + i * kRPI + row_in;
+    for (int u = 0; u < kRuns; ++u) {
+      const int fr = row0 + u * kRunStride + kRun * grp;
+      const int lp = fr / bpp;
+      const int rin = fr - lp * bpp;
       const int j = lp - lp0;
       int pg = __shfl_sync(0xffffffffu, pg_lane, j & 31);
-      if (j >= 32) {  // item spans more than 32 pages (tiny pages): direct lookup
+      if (j >= 32) {  // item spans more than 32 pages (small pages): direct lookup
         pg = (lp < p.c.max_pages_per_req) ? p.c.block_table[(long long)r * p.c.max_pages_per_req + lp] : -1;
         if (pg >= p.c.num_pages) pg = -1;
       }
-      v[i] = make_uint4(0, 0, 0, 0);
-      h[i] = 0u;
-      if (row < n) {
+      hv[u] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int t = 0; t < kRun; ++t) v[u * kRun + t] = make_uint4(0, 0, 0, 0);
+      if (fr < n) {
         if (pg >= 0) {
           const uint8_t *pb = p.c.kc + (long long)pg * page_bytes;
-          v[i] = scan_load(reinterpret_cast<const uint4 *>(pb + (long long)off * DI + sub * 16), pol_stream);
-          h[i] = scan_load32(
-              reinterpret_cast<const uint32_t *>(pb + lo_bytes + (long long)off * kHiRow + sub * 4),
+#pragma unroll
+          for (int t = 0; t < kRun; ++t)
+            if (fr + t < n)
+              v[u * kRun + t] = scan_load(
+                  reinterpret_cast<const uint4 *>(pb + (long long)(rin + t) * DI + sub * 16), pol_stream);
+          hv[u] = scan_load(
+              reinterpret_cast<const uint4 *>(pb + lo_bytes + 4LL * ((long long)sub * bpp + rin)),
               pol_stream);
-        } else if (lane == 0 || sub == 0) {
+        } else if (sub == 0) {
           record_error(kErrBounds);
         }
       }
-      off += kRPI;
-      while (off >= bpp) {
-        off -= bpp;
-        ++lp;
-      }
-    }
     }
     // prefetch the next item's block-table entries
     it += nwarps;
@@ -798,14 +764,17 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
     int acc[16];
 #pragma unroll
     for (int i = 0; i < kItemLoads; ++i) {
+      const uint4 hw4 = hv[i / kRun];
+      const int t = i % kRun;
+      const uint32_t h = t == 0 ? hw4.x : t == 1 ? hw4.y : t == 2 ? hw4.z : hw4.w;
       int a = dp4a_us(v[i].x, q[0], 0);
       a = dp4a_us(v[i].y, q[1], a);
       a = dp4a_us(v[i].z, q[2], a);
       a = dp4a_us(v[i].w, q[3], a);
-      int b = dp4a_us(h[i] & 0x03030303u, q[0], 0);
-      b = dp4a_us((h[i] >> 2) & 0x03030303u, q[1], b);
-      b = dp4a_us((h[i] >> 4) & 0x03030303u, q[2], b);
-      b = dp4a_us((h[i] >> 6) & 0x03030303u, q[3], b);
+      int b = dp4a_us(h & 0x03030303u, q[0], 0);
+      b = dp4a_us((h >> 2) & 0x03030303u, q[1], b);
+      b = dp4a_us((h >> 4) & 0x03030303u, q[2], b);
+      b = dp4a_us((h >> 6) & 0x03030303u, q[3], b);
       acc[i] = a + (b << 8);
     }
     reduce_scatter16<kLPR>(acc, lane);
@@ -813,7 +782,7 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
 #pragma unroll
     for (int k = 0; k < kVals; ++k) {
       const int i = ((lane % kLPR) << (4 - kR)) | k;
-      const int row = row0 + i * kRPI + row_in;
+      const int row = row0 + (i / kRun) * kRunStride + kRun * grp + (i % kRun);
       if (row < n) score_store(sc + row, acc[k] + qbias, pol_keep);
     }
     if (!more) break;

@@ -323,7 +323,7 @@ const char *qsa_status_string(int32_t status) {
 int32_t qsa_abi_version(void) { return 2; }
 
 size_t qsa_kc_page_bytes(int32_t page_size, int32_t idx_dim) {
-  if (page_size <= 0 || page_size % 4 != 0) return 0;
+  if (page_size <= 0 || page_size % 16 != 0) return 0;
   if (idx_dim != 32 && idx_dim != 64 && idx_dim != 128) return 0;
   return (size_t)qsa::kc_page_bytes(page_size, idx_dim);
 }
@@ -337,6 +337,7 @@ qsa_status qsa_compress_append(const qsa_cache *cache, int32_t B, const int32_t 
   if (B == 0 || max_new_per_req == 0) return QSA_OK;
   if (B > cache->ring_rows || B > 65535) return QSA_ERR_INVALID_ARG;
   if (!pos0 || !cu_new || !k_new || !cache->kc || !cache->ring) return QSA_ERR_INVALID_ARG;
+  if (cache->page_size % 16 != 0) return QSA_ERR_UNSUPPORTED;  // packed compressed-key pages
   if (!aligned(k_new, 4) || !aligned(cache->kc, 16) || !aligned(cache->ring, 4))
     return QSA_ERR_INVALID_ARG;
   const long long max_blocks = (long long)max_new_per_req / 4 + 2;
@@ -381,6 +382,7 @@ qsa_status index_topk_call(const qsa_cache *cache, int32_t B, const int8_t *q_id
   if (!q_idx || !ctx_lens || !(sel || tokens) || !workspace || !cache->kc) return QSA_ERR_INVALID_ARG;
   if (cache->idx_dim != 32 && cache->idx_dim != 64 && cache->idx_dim != 128)
     return QSA_ERR_UNSUPPORTED;
+  if (cache->page_size % 16 != 0) return QSA_ERR_UNSUPPORTED;  // packed compressed-key pages
   if (!aligned(cache->kc, 16) || !aligned(q_idx, 4) || !aligned(workspace, 16) ||
       (scores && !aligned(scores, 4)) || (tokens && !aligned(tokens, 16)))
     return QSA_ERR_INVALID_ARG;
@@ -658,6 +660,7 @@ qsa_status qsa_index_topk_noalloc(const qsa_cache *cache, int32_t B, const int8_
   if (!q_idx || !ctx_lens || !sel || !cache->kc) return QSA_ERR_INVALID_ARG;
   if (cache->idx_dim != 32 && cache->idx_dim != 64 && cache->idx_dim != 128)
     return QSA_ERR_UNSUPPORTED;
+  if (cache->page_size % 16 != 0) return QSA_ERR_UNSUPPORTED;  // packed compressed-key pages
   if (!aligned(cache->kc, 16) || !aligned(q_idx, 4)) return QSA_ERR_INVALID_ARG;
   int32_t *scores = noalloc_scores_ptr();
   if (!scores) return QSA_ERR_CUDA;

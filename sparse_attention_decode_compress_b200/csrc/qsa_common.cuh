@@ -78,14 +78,16 @@ __host__ __device__ __forceinline__ long long ceil_div_ll(long long a, long long
   return (a + b - 1) / b;
 }
 
-// Packed compressed-key page (P tokens, indexer dim d): a key value v of a
-// micro-block (a sum of 4 int8 keys, |v| <= 508) is stored as its low byte
-// v & 255 and a 2-bit high field (v >> 8) + 2 in [0, 3], so v =
-// 256 * (field - 2) + low byte.  A page holds the P/4 rows of d low bytes,
-// then the P/4 rows of d/4 high-field bytes, then padding to 16 bytes.  In
-// the high row, dims 16w .. 16w+15 form 32-bit word w (little endian):
-// dim 16w + 4s + k sits at bits 8k + 2s, so (word >> 2s) & 0x03030303 holds
-// the fields of dims 16w + 4s .. 16w + 4s + 3 in its four bytes.
+// Packed compressed-key page (P tokens, R = P/4 micro-block rows, indexer
+// dim d): a key value v (a sum of 4 int8 keys, -512 <= v <= 508) is stored
+// as its low byte v & 255 and a 2-bit high field (v >> 8) + 2 in [0, 3], so
+// v = 256 * (field - 2) + low byte.  A page holds the R rows of d low bytes,
+// then the high fields as 32-bit words, then padding to 16 bytes.  Word
+// (w, row) holds the fields of dims 16w .. 16w+15 of a row and sits at word
+// index w * R + row of the high part (dim-group major, so four consecutive
+// rows of one dim group are 16 contiguous bytes); dim 16w + 4s + k is at bits
+// 8k + 2s, so (word >> 2s) & 0x03030303 holds the fields of dims
+// 16w + 4s .. 16w + 4s + 3 in its four bytes.
 __host__ __device__ __forceinline__ long long kc_lo_bytes(int page_size, int d) {
   return (long long)(page_size / 4) * d;
 }

@@ -123,12 +123,14 @@ def oracle_request(batch: QSABatch, r: int, num_splits: int) -> dict:
 def unpack_kc_pages(pages: np.ndarray, P: int, d: int) -> np.ndarray:
     """Compressed-key values [n, P/4, d] (int64) of packed pages [n, bytes],
     read by the layout include/qsa.h states at qsa_kc_page_bytes: R = P/4
-    rows of d low bytes, then R rows of d/4 high-field bytes, dim 16w+4s+k
-    of a row at bits 8k+2s of its 32-bit word w; value = 256*(field-2)+low."""
+    rows of d low bytes, then 32-bit field words, word w*R + row holding
+    dims 16w..16w+15 of the row, dim 16w+4s+k at bits 8k+2s; value =
+    256*(field-2)+low."""
     R = P // 4
     n = pages.shape[0]
     lo = pages[:, :R * d].reshape(n, R, d).astype(np.int64)
-    hib = pages[:, R * d:R * d + R * d // 4].reshape(n, R, d // 16, 4).astype(np.int64)
+    hib = pages[:, R * d:R * d + R * d // 4].reshape(n, d // 16, R, 4).transpose(0, 2, 1, 3)
+    hib = hib.astype(np.int64)
     s = np.arange(4)
     f = (hib[:, :, :, None, :] >> (2 * s)[:, None]) & 3   # [n, R, w, s, k]
     return 256 * (f.reshape(n, R, d) - 2) + lo

@@ -19,11 +19,11 @@ def _pack(vals: np.ndarray, P: int, d: int, page_bytes: int) -> np.ndarray:
                 out[pg, row * d + j] = v & 255
                 f = (v >> 8) + 2
                 w, s, k = j // 16, (j % 16) // 4, j % 4
-                out[pg, R * d + row * (d // 4) + 4 * w + k] |= f << (2 * s)
+                out[pg, R * d + 4 * (w * R + row) + k] |= f << (2 * s)
     return out
 
 
-@pytest.mark.parametrize("P,d", [(64, 128), (16, 32), (64, 64), (4, 32), (16, 128)])
+@pytest.mark.parametrize("P,d", [(64, 128), (16, 32), (64, 64), (32, 32), (16, 128)])
 def test_page_bytes(P, d):
     lib = _lib.load()
     R = P // 4
@@ -34,11 +34,12 @@ def test_page_bytes(P, d):
 def test_page_bytes_rejects_bad_geometry():
     lib = _lib.load()
     assert lib.qsa_kc_page_bytes(6, 128) == 0
+    assert lib.qsa_kc_page_bytes(8, 128) == 0   # pages hold whole 4-row runs: P % 16 == 0
     assert lib.qsa_kc_page_bytes(64, 48) == 0
     assert lib.qsa_kc_page_bytes(0, 128) == 0
 
 
-@pytest.mark.parametrize("P,d", [(64, 128), (16, 32), (8, 64)])
+@pytest.mark.parametrize("P,d", [(64, 128), (16, 32), (32, 64)])
 def test_harness_reader_round_trip(P, d):
     lib = _lib.load()
     rng = np.random.default_rng(P * d)
