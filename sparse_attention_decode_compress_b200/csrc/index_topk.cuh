@@ -626,6 +626,10 @@ __device__ __forceinline__ void score_store(int32_t *p, int v, uint64_t policy) 
   asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(policy) : "memory");
 #endif
 }
+__device__ __forceinline__ void score_store2(int32_t *p, int a, int b, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v2.b32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(a), "r"(b), "l"(policy)
+               : "memory");
+}
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
@@ -778,12 +782,21 @@ __global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_ke
       acc[i] = a + (b << 8);
     }
     reduce_scatter16<kLPR>(acc, lane);
+    // values k, k+1 of a lane are consecutive rows (load indices 2m, 2m+1
+    // of one run): one 8-byte store where aligned, so a warp's stores fill
+    // whole sectors of the score row
     int32_t *sc = p.scores + (long long)r * p.max_blocks;
 #pragma unroll
-    for (int k = 0; k < kVals; ++k) {
+    for (int k = 0; k < kVals; k += 2) {
       const int i = ((lane % kLPR) << (4 - kR)) | k;
       const int row = row0 + (i / kRun) * kRunStride + kRun * grp + (i % kRun);
-      if (row < n) score_store(sc + row, acc[k] + qbias, pol_keep);
+      int32_t *dst = sc + row;
+      if (row + 1 < n && (reinterpret_cast<uintptr_t>(dst) & 7u) == 0) {
+        score_store2(dst, acc[k] + qbias, acc[k + 1] + qbias, pol_keep);
+      } else {
+        if (row < n) score_store(dst, acc[k] + qbias, pol_keep);
+        if (row + 1 < n) score_store(dst + 1, acc[k + 1] + qbias, pol_keep);
+      }
     }
     if (!more) break;
   }
