@@ -528,13 +528,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
 }
 
 // ------------------------------------------------------------- the scan --
-// Persistent warps stream the compressed keys straight into registers with
-// 16-byte loads: an item is 8 KiB of one request (16 loads per lane, all in
-// flight together), i.e. 4096/d rows; lane l reads dims 8*(l % LPR) .. +7 of
-// row (i * RPI + l / LPR) for load i.  Plain loads beat a shared-memory ring
-// fed by bulk copies here (measured on this GPU: ~7.0 vs ~3.9 TB/s on
-// randomly permuted 4 KiB pages).  The block-table entries of the next item
-// are fetched while the current one computes.
+// Persistent warps stream the packed compressed keys straight into registers
+// with 16-byte loads: an item is 8192/d rows of one request (8 KiB of low
+// bytes plus their high fields: 20 loads per lane, all in flight together).
+// Lane l owns dims 16*(l % LPR) .. +15 of its rows, which come in runs of 4
+// consecutive rows (one 16-byte load of the run's high-field words).  Plain
+// loads beat a shared-memory ring fed by bulk copies here (measured on this
+// GPU: ~7.0 vs ~3.9 TB/s on randomly permuted 4 KiB pages).  The block-table
+// entries of the next item are fetched while the current one computes.
 
 constexpr int kScanThreads = 128;
 constexpr int kItemLoads = 16;  // 16-byte key loads per lane per item (8 KiB of low bytes per warp)
@@ -591,40 +592,23 @@ struct ItemWalker {
   }
 };
 
-#ifndef QSA_SCAN_MIN_CTAS
-#define QSA_SCAN_MIN_CTAS 4
-#endif
-#ifndef QSA_SCAN_LOAD
-#define QSA_SCAN_LOAD 2
-#endif
-#ifndef QSA_SCORE_STORE
-#define QSA_SCORE_STORE 1
-#endif
-// 16-byte load of compressed keys, read once per call.
+// 4 CTAs of 128 threads per SM: 118 registers, no spills (at 5 the packed
+// scan spilled and ran 2.5 % slower).
+constexpr int kScanMinCtas = 4;
+// 16-byte load of compressed keys, read once per call: not cached in L1, L2
+// evict-first (the stream does not push the scores out of L2), 256-byte L2
+// prefetch.
 __device__ __forceinline__ uint4 scan_load(const uint4 *p, uint64_t policy) {
   uint4 v;
-#if QSA_SCAN_LOAD == 0
-  v = __ldcs(p);
-#elif QSA_SCAN_LOAD == 1
-  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-#else
-  // not cached in L1, L2 evict-first (the stream does not push the scores out
-  // of L2), 256-byte L2 prefetch
   asm volatile(
       "ld.global.nc.L1::no_allocate.L2::cache_hint.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
       : "l"(p), "l"(policy));
-#endif
   return v;
 }
-// Score store; L2 evict-last keeps it for the selection kernel.
+// Score stores; L2 evict-last keeps them for the selection kernel.
 __device__ __forceinline__ void score_store(int32_t *p, int v, uint64_t policy) {
-#if QSA_SCORE_STORE == 0
-  *p = v;
-#else
   asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(policy) : "memory");
-#endif
 }
 __device__ __forceinline__ void score_store2(int32_t *p, int a, int b, uint64_t policy) {
   asm volatile("st.global.L2::cache_hint.v2.b32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(a), "r"(b), "l"(policy)
@@ -655,7 +639,7 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
 // the first two by dp4a (unsigned key bytes, signed query bytes), the last a
 // constant of the request.
 template <int DI, int BPPC>
-__global__ void __launch_bounds__(kScanThreads, QSA_SCAN_MIN_CTAS) index_scan_kernel(Params p) {
+__global__ void __launch_bounds__(kScanThreads, kScanMinCtas) index_scan_kernel(Params p) {
   pdl_open();
   static_assert(DI == 32 || DI == 64 || DI == 128, "indexer dim");
   constexpr int kLPR = DI / 16;                   // lanes per row (16 dims each)

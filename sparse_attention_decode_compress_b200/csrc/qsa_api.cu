@@ -185,34 +185,16 @@ int decode_chunk_blocks(int B, int Hkv, int topk, int S, int S_active, long long
   return std::max(chunk, qsa::dec::kMinChunkBlocks);
 }
 
-// Worker warps per SM and ring depth of the tensor-core decode kernel: as
-// many warps as registers allow (query-row tiles NT set the accumulator
-// size), then as deep a ring as shared memory allows.
-#ifndef QSA_DEC_NW_BF16
-#define QSA_DEC_NW_BF16 12
-#endif
-#ifndef QSA_DEC_NS_BF16
-#define QSA_DEC_NS_BF16 2
-#endif
-// fp8: 12 warps with a 2-stage ring beat 8 warps with 4 stages (decode of
-// the mixed fp8 batch 325 -> 268 us): the fp8 path is bound by per-chunk
-// latency, not by bytes in flight.
-#ifndef QSA_DEC_NW_FP8
-#define QSA_DEC_NW_FP8 12
-#endif
-#ifndef QSA_DEC_NS_FP8
-#define QSA_DEC_NS_FP8 2
-#endif
-template <int D, int NT, bool FP8>
-struct DecodeShape {
-  static constexpr int NW = (!FP8 && NT <= 2) ? QSA_DEC_NW_BF16 : (FP8 ? QSA_DEC_NW_FP8 : 8);
-  static constexpr int NS = (!FP8 && NT <= 2) ? QSA_DEC_NS_BF16 : (FP8 ? QSA_DEC_NS_FP8 : 3);
-};
-
+// Worker warps per SM and ring depth of the persistent warp decode (8 query
+// rows per kv head): 12 warps (166 registers, bf16) with a 2-stage ring.
+// fp8: 3 or 4 stages (its stages are half the bytes) measured 1.5-3 % slower
+// than 2, and 8 warps with 4 stages slower than 12 with 2.
+constexpr int kDecWarps = 12;
+constexpr int kDecStages = 2;
 template <int D, int NT, bool FP8>
 qsa_status launch_decode_warp(qsa::dec::Params p, cudaStream_t stream) {
-  constexpr int NW = DecodeShape<D, NT, FP8>::NW;
-  constexpr int NS = DecodeShape<D, NT, FP8>::NS;
+  constexpr int NW = kDecWarps;
+  constexpr int NS = kDecStages;
   static bool done[kMaxDevices] = {false};
   static int blocks_per_sm[kMaxDevices] = {0};
   auto kernel = qsa::dec::sparse_decode_warp_kernel<D, NT, FP8, NW, NS>;

@@ -31,10 +31,7 @@ namespace dec {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-#ifndef QSA_CHUNK_BLOCKS
-#define QSA_CHUNK_BLOCKS 128
-#endif
-constexpr int kChunkBlocks = QSA_CHUNK_BLOCKS;  // capacity of a work item, micro-blocks
+constexpr int kChunkBlocks = 128;  // largest chunk the host picks (bf16 metadata piece), micro-blocks
 constexpr int kChunkTokens = kChunkBlocks * 4;
 constexpr int kMinChunkBlocks = 32;  // smallest chunk the host picks
 constexpr int kMaxSplits = 16;
