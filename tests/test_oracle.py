@@ -174,7 +174,8 @@ def test_compress_one_hot_locality():
         assert kc[t // 4, 1] == 7
 
 
-def test_compress_extremes_fit_int16():
+def test_compress_extremes_fit_ten_bits():
+    # the range the packed 10-bit cache layout must hold: [-512, 508]
     k = np.full((8, 4), -128, dtype=np.int8)
     assert ref.compress_keys(k).min() == -512
     k = np.full((8, 4), 127, dtype=np.int8)
