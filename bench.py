@@ -117,9 +117,32 @@ def algorithmic_bytes(w, L: int, num_splits: int) -> dict:
                 total=idx + dec + merge + append)
 
 
+L2_BYTES = 126 * 1000 * 1000  # B200 L2
+
+
+def mean_context(w) -> float:
+    """Mean context length of the workload's length distribution."""
+    kind, *a = w.ctx.split(":")
+    if kind == "fixed":
+        return float(a[0])
+    lo, hi = float(a[0]), float(a[1])
+    if kind == "uniform":
+        return (lo + hi) / 2
+    return (hi - lo) / math.log(hi / lo)  # loguniform
+
+
+def step_bytes(w, num_splits: int) -> int:
+    """Algorithmic bytes of one step of the whole batch at the mean length."""
+    return int(w.batch * algorithmic_bytes(w, int(mean_context(w)), num_splits)["total"])
+
+
 def workload_config(w, num_splits: int, world: int, dcp: bool = False) -> dict:
     """The `config` object of the JSON line (both arms)."""
     kind, *a = w.ctx.split(":")
+    sb = step_bytes(w, num_splits)
+    l2 = (f"inputs larger than L2: ~{sb / 1e9:.2f} GB read per step (mostly packed "
+          f"compressed keys), no flush" if sb > L2_BYTES else
+          f"inputs smaller than L2 (~{sb / 1e6:.0f} MB per step), no flush: steps may hit L2")
     par = "single GPU"
     if world > 1:
         par = f"decode context parallel x{world} (NCCL all-gather)" if dcp else f"replicas x{world}"
@@ -128,7 +151,7 @@ def workload_config(w, num_splits: int, world: int, dcp: bool = False) -> dict:
             "seq_len": int(a[-1]), "query_tokens": w.T, "kv_splits": num_splits,
             "topk_blocks": w.topk, "page_size": w.page_size,
             "parallelism": par,
-            "l2": "inputs larger than L2 (2 GiB compressed keys read per step)",
+            "l2": l2,
             "timing": "value: K back-to-back steps (one CUDA graph of the K steps, replayed "
                       "once after an untimed replay; --no-graph: eager launches); kernel_ms and "
                       "roofline: a second, eager K-step pass with events between the kernels"}
