@@ -235,6 +235,12 @@ size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32
  *     o_s   = sum_{i in split} exp(logit_i - lse_s) v_i,
  * and an empty split writes o_s = 0, lse_s = -inf.  FP8 K/V values are
  * code * scale[page][kv head].
+ * Numerics: products on tensor cores with fp32 accumulation (bf16 caches:
+ * bf16 operands; fp8 caches: f16 operands, which hold every E4M3 code
+ * exactly, with Q scaled into f16 range by a power of two per row); the
+ * softmax weights enter the value product as a hi + lo pair; fp32 caches
+ * run in fp32.  Outputs stay within 1e-2 absolute and 2e-3 relative L2 (o)
+ * and 1e-4 (lse) of the exact result.
  *
  *   q        [B, T, Hq, D] of q_dtype (QSA_F32 or QSA_BF16; BF16 for
  *            BF16/FP8 caches, F32 for F32 caches)
