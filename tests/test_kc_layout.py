@@ -48,3 +48,19 @@ def test_harness_reader_round_trip(P, d):
     vals[0, 0, 4:8] = [255, 256, -256, -257]
     pages = _pack(vals, P, d, int(lib.qsa_kc_page_bytes(P, d)))
     assert np.array_equal(H.unpack_kc_pages(pages, P, d), vals)
+
+
+def test_cache_allocation_uses_the_packed_page():
+    import torch
+    from sparse_attention_decode_compress_b200 import QSACache
+    k = torch.zeros((5, 64, 2, 128), dtype=torch.bfloat16)
+    bt = torch.zeros((1, 5), dtype=torch.int32)
+    c = QSACache.allocate(k, k.clone(), bt, idx_dim=128, ring_rows=1)
+    assert c.kc.dtype == torch.uint8 and tuple(c.kc.shape) == (5, 16 * 128 + 16 * 32)
+    k8 = torch.zeros((5, 8, 2, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="unsupported compressed-key geometry"):
+        QSACache.allocate(k8, k8.clone(), bt, idx_dim=128, ring_rows=1)
+    # an int16-shaped cache is rejected before any pointer is taken
+    bad = QSACache(k, k.clone(), torch.zeros((5, 4096), dtype=torch.uint8), c.ring, bt)
+    with pytest.raises(ValueError, match="qsa_kc_page_bytes"):
+        bad.struct()
