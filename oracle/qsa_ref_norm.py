@@ -24,6 +24,10 @@ With floating-point scores a CUDA path and this oracle can order blocks whose
 scores differ by rounding differently, so parity is stated by
 ``selection_within_tolerance``: the kept set must be a top-k of the oracle's
 scores up to a tolerance at the threshold.
+
+Pins: ``tests/test_oracle_norm.py`` checks every function against closed
+forms, the integer oracle (mean x 4 = sum on full blocks), torch's RMS norm
+and brute force.
 """
 from __future__ import annotations
 
