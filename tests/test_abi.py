@@ -103,3 +103,14 @@ def test_bad_sizes_rejected_on_host():
     assert lib.qsa_lse_merge(2, 0, 4, None, None, None, None, None) == 0
     assert lib.qsa_index_topk(ctypes.byref(c), 0, None, None, None, 16, 8, None, None, None, 0,
                               None) == 0
+
+
+def test_page_sizes_off_the_packed_key_runs_are_unsupported():
+    # P = 8 is a multiple of the compress ratio but not of 16: the packed
+    # compressed-key pages are read in runs of 4 micro-blocks
+    lib = _lib.load()
+    c = _cache(page_size=8)
+    assert lib.qsa_compress_append(ctypes.byref(c), 1, 0x100, 0x100, 0x100, 1, None) == 2
+    assert lib.qsa_index_topk(ctypes.byref(c), 1, 0x100, 0x100, None, 16, 8, 0x100, None, 0x100,
+                              1 << 20, None) == 2
+    assert lib.qsa_kc_page_bytes(8, 128) == 0
