@@ -64,8 +64,8 @@ typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype;
  * block-table entry names the same physical page in all of them. */
 typedef struct {
   int32_t num_pages;    /* physical pages in each cache                       */
-  int32_t page_size;    /* tokens per page P; multiple of 16 (4-token micro-
-                           blocks, packed compressed keys in runs of 4)      */
+  int32_t page_size;    /* tokens per page P; a multiple of the compress
+                           ratio 4 (whole 4-token micro-blocks per page)     */
   int32_t num_kv_heads; /* Hkv                                                */
   int32_t head_dim;     /* D: 64 or 128                                       */
   int32_t idx_dim;      /* indexer dim d: 32, 64 or 128                       */
@@ -93,9 +93,8 @@ int32_t qsa_abi_version(void);
 
 /*
  * qsa_kc_page_bytes — bytes of one page of the packed compressed-key cache,
- * or 0 for an unsupported geometry (page_size not a positive multiple of 16,
- * idx_dim not 32, 64 or 128).  qsa_compress_append and qsa_index_topk return
- * QSA_ERR_UNSUPPORTED for a page_size that is not a multiple of 16.
+ * or 0 for an unsupported geometry (page_size not a positive multiple of 4,
+ * idx_dim not 32, 64 or 128).
  *
  * A compressed key value v of micro-block b, dim j (the sum of 4 int8 keys,
  * -512 <= v <= 508) is stored losslessly in 10 bits: its low byte v & 255
@@ -136,8 +135,9 @@ size_t qsa_kc_page_bytes(int32_t page_size, int32_t idx_dim);
  * are read back from ring row r).  A decode step passes T new tokens per
  * request; a prefill passes whole chunks (complete blocks are pooled
  * straight from k_new).  Errors: QSA_ERR_INVALID_ARG for null pointers,
- * B < 0, B > ring_rows or page_size % 4 != 0; QSA_ERR_UNSUPPORTED for
- * page_size % 16 != 0 or an unsupported idx_dim.
+ * B < 0, B > ring_rows or page_size % 4 != 0 (PR #53896 report, 实现拆解:
+ * the block size must be divisible by the compress ratio);
+ * QSA_ERR_UNSUPPORTED for an unsupported idx_dim.
  */
 qsa_status qsa_compress_append(const qsa_cache *cache, int32_t B, const int32_t *pos0,
                                const int32_t *cu_new, const int8_t *k_new,
@@ -251,9 +251,11 @@ size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32
  *   o_part   [S, B, T, Hq, D] float32 output
  *   lse_part [S, B, T, Hq] float32 output (natural log)
  *   workspace  >= qsa_sparse_decode_workspace_bytes(...), 16-byte aligned,
- *            ZERO-FILLED before first use and left zeroed by every completed
- *            call: its header holds the work counter and the per-split
- *            tickets; the rest holds chunk partials.
+ *            any contents: its header holds the work counter and the
+ *            per-split tickets, which the call zeroes itself (a one-CTA
+ *            kernel ahead of the decode kernel); the rest holds chunk
+ *            partials.  Calls that overlap on the GPU need separate
+ *            workspaces.
  * Errors: QSA_ERR_INVALID_ARG / QSA_ERR_UNSUPPORTED on the host
  * (QSA_ERR_UNSUPPORTED also when num_pages * page_size * Hkv exceeds
  * 2^31 - 1 cache rows); page or position violations -> QSA_ERR_BOUNDS on the
@@ -353,7 +355,10 @@ qsa_status qsa_lse_merge(int32_t num_splits, int64_t rows, int32_t D, const floa
  * stream capture.  All calls share the array: calls that overlap on the GPU
  * (two streams, or two devices' threads racing on the same device) race on
  * it; calls in order on one stream do not.  QSA_ERR_CUDA if the address
- * lookup fails.
+ * lookup fails.  The looked-up address is kept for the life of the process,
+ * so after cudaDeviceReset on a device this entry point must not be called
+ * on that device again in the same process.  Each call's scan writes every
+ * score its selection reads, so the array needs no clearing between calls.
  */
 qsa_status qsa_index_topk_noalloc(const qsa_cache *cache, int32_t B, const int8_t *q_idx,
                                   const int32_t *ctx_lens, const int32_t *n_sel,

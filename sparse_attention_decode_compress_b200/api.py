@@ -125,7 +125,8 @@ def qsa_sparse_decode_workspace_bytes(B: int, T: int, Hq: int, Hkv: int, D: int,
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:
-    """Zero-filled workspace (the counters at its start must begin at zero)."""
+    """Workspace buffer (zero-filled; no call needs it zeroed: the decode
+    zeroes its own header in every call)."""
     return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
 
 

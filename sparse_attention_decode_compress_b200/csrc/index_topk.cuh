@@ -606,6 +606,15 @@ __device__ __forceinline__ uint4 scan_load(const uint4 *p, uint64_t policy) {
       : "l"(p), "l"(policy));
   return v;
 }
+// 4-byte load of one row's high-field word (pages whose rows do not come in
+// aligned runs of 4), same caching as scan_load.
+__device__ __forceinline__ uint32_t scan_load32(const uint32_t *p, uint64_t policy) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.b32 %0, [%1], %2;"
+               : "=r"(v)
+               : "l"(p), "l"(policy));
+  return v;
+}
 // Score stores; L2 evict-last keeps them for the selection kernel.
 __device__ __forceinline__ void score_store(int32_t *p, int v, uint64_t policy) {
   asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(policy) : "memory");
@@ -628,7 +637,9 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
 }
 
 // BPPC: micro-blocks per page when it is a compile-time constant (16 for
-// 64-token pages, 4 for 16-token pages), 0 for any page size.
+// 64-token pages, 4 for 16-token pages), 0 for any other multiple of 4
+// micro-blocks per page, -1 for pages of 4, 8 or 12 mod 16 tokens (the
+// rows of a run may then cross a page: each row is looked up alone).
 //
 // Keys are the packed pages of qsa_common.cuh.  A lane owns 16 dims of its
 // rows, which come in runs of 4 consecutive rows: per run, four 16-byte
@@ -710,34 +721,75 @@ __global__ void __launch_bounds__(kScanThreads, kScanMinCtas) index_scan_kernel(
     // invalid page is skipped (scores garbage, error recorded)
     uint4 v[kItemLoads];
     uint4 hv[kRuns];
-#pragma unroll
-    for (int u = 0; u < kRuns; ++u) {
-      const int fr = row0 + u * kRunStride + kRun * grp;
-      const int lp = fr / bpp;
-      const int rin = fr - lp * bpp;
+    // physical page of logical page lp of request r (lp in [lp0, ...)): from
+    // the lane that fetched it, or looked up directly when the item spans
+    // more than 32 pages (small pages)
+    auto page_of = [&](int lp) -> int {
       const int j = lp - lp0;
       int pg = __shfl_sync(0xffffffffu, pg_lane, j & 31);
-      if (j >= 32) {  // item spans more than 32 pages (small pages): direct lookup
+      if (j >= 32) {
         pg = (lp < p.c.max_pages_per_req) ? p.c.block_table[(long long)r * p.c.max_pages_per_req + lp] : -1;
         if (pg >= p.c.num_pages) pg = -1;
       }
-      hv[u] = make_uint4(0, 0, 0, 0);
+      return pg;
+    };
+    if constexpr (BPPC >= 0) {
 #pragma unroll
-      for (int t = 0; t < kRun; ++t) v[u * kRun + t] = make_uint4(0, 0, 0, 0);
-      if (fr < n) {
-        if (pg >= 0) {
-          const uint8_t *pb = p.c.kc + (long long)pg * page_bytes;
+      for (int u = 0; u < kRuns; ++u) {
+        const int fr = row0 + u * kRunStride + kRun * grp;
+        const int lp = fr / bpp;
+        const int rin = fr - lp * bpp;
+        const int pg = page_of(lp);
+        hv[u] = make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int t = 0; t < kRun; ++t)
-            if (fr + t < n)
-              v[u * kRun + t] = scan_load(
-                  reinterpret_cast<const uint4 *>(pb + (long long)(rin + t) * DI + sub * 16), pol_stream);
-          hv[u] = scan_load(
-              reinterpret_cast<const uint4 *>(pb + lo_bytes + 4LL * ((long long)sub * bpp + rin)),
-              pol_stream);
-        } else if (sub == 0) {
-          record_error(kErrBounds);
+        for (int t = 0; t < kRun; ++t) v[u * kRun + t] = make_uint4(0, 0, 0, 0);
+        if (fr < n) {
+          if (pg >= 0) {
+            const uint8_t *pb = p.c.kc + (long long)pg * page_bytes;
+#pragma unroll
+            for (int t = 0; t < kRun; ++t)
+              if (fr + t < n)
+                v[u * kRun + t] = scan_load(
+                    reinterpret_cast<const uint4 *>(pb + (long long)(rin + t) * DI + sub * 16), pol_stream);
+            hv[u] = scan_load(
+                reinterpret_cast<const uint4 *>(pb + lo_bytes + 4LL * ((long long)sub * bpp + rin)),
+                pol_stream);
+          } else if (sub == 0) {
+            record_error(kErrBounds);
+          }
         }
+      }
+    } else {
+      // pages of 4, 8 or 12 mod 16 tokens: the rows of a run may sit on two
+      // pages and their high-field words are not 16-byte aligned, so each
+      // row is looked up and loaded on its own (16 bytes of low bytes and
+      // one 4-byte field word)
+#pragma unroll
+      for (int u = 0; u < kRuns; ++u) {
+        const int fr = row0 + u * kRunStride + kRun * grp;
+        uint32_t h[kRun];
+#pragma unroll
+        for (int t = 0; t < kRun; ++t) {
+          const int row = fr + t;
+          const int lp = row / bpp;
+          const int rin = row - lp * bpp;
+          const int pg = page_of(lp);
+          v[u * kRun + t] = make_uint4(0, 0, 0, 0);
+          h[t] = 0u;
+          if (row < n) {
+            if (pg >= 0) {
+              const uint8_t *pb = p.c.kc + (long long)pg * page_bytes;
+              v[u * kRun + t] = scan_load(
+                  reinterpret_cast<const uint4 *>(pb + (long long)rin * DI + sub * 16), pol_stream);
+              h[t] = scan_load32(
+                  reinterpret_cast<const uint32_t *>(pb + lo_bytes + 4LL * ((long long)sub * bpp + rin)),
+                  pol_stream);
+            } else if (sub == 0) {
+              record_error(kErrBounds);
+            }
+          }
+        }
+        hv[u] = make_uint4(h[0], h[1], h[2], h[3]);
       }
     }
     // prefetch the next item's block-table entries

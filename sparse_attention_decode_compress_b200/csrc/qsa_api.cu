@@ -23,9 +23,10 @@ namespace {
 using qsa::CacheDev;
 
 constexpr size_t kAlign = 256;
-// Both workspaces start with this many bytes of completion counters, which
-// must be zero before the first call and are left zero by every completed
-// call (the layout does not depend on the call's sizes).
+// Both workspaces start with a header of this many bytes (the layout does
+// not depend on the call's sizes).  The decode keeps its work counters and
+// split tickets there and zeroes them at the start of every call; the
+// indexer leaves it unused.
 constexpr size_t kTicketBytes = 64 * 1024;
 constexpr int kMaxDevices = 64;
 
@@ -150,6 +151,25 @@ qsa_status launch_index_topk(const qsa::topk::Params &p, cudaStream_t stream) {
   qsa_status st = launch(true, kernel, dim3(grid), dim3(kScanThreads), 0, stream, p);
   if (st != QSA_OK) return st;
   return launch(true, select_kernel, dim3(p.B), dim3(kSelThreads), select_smem(), stream, p);
+}
+
+// Scan instance for the indexer dim and page geometry: constant page
+// geometry for 64- and 16-token pages, any multiple of 16 tokens, and pages
+// of 4, 8 or 12 mod 16 tokens (rows of a run may cross a page).
+template <int DI>
+qsa_status dispatch_index_topk_d(const qsa::topk::Params &p, int P, cudaStream_t s) {
+  if (P == 64) return launch_index_topk<DI, 16>(p, s);
+  if (P == 16) return launch_index_topk<DI, 4>(p, s);
+  if (P % 16 == 0) return launch_index_topk<DI, 0>(p, s);
+  return launch_index_topk<DI, -1>(p, s);
+}
+
+qsa_status dispatch_index_topk(const qsa::topk::Params &p, int idx_dim, int P, cudaStream_t s) {
+  switch (idx_dim) {
+    case 32: return dispatch_index_topk_d<32>(p, P, s);
+    case 64: return dispatch_index_topk_d<64>(p, P, s);
+    default: return dispatch_index_topk_d<128>(p, P, s);
+  }
 }
 
 // ---------------------------------------------------------------- decode --
@@ -305,7 +325,7 @@ const char *qsa_status_string(int32_t status) {
 int32_t qsa_abi_version(void) { return 2; }
 
 size_t qsa_kc_page_bytes(int32_t page_size, int32_t idx_dim) {
-  if (page_size <= 0 || page_size % 16 != 0) return 0;
+  if (page_size <= 0 || page_size % 4 != 0) return 0;
   if (idx_dim != 32 && idx_dim != 64 && idx_dim != 128) return 0;
   return (size_t)qsa::kc_page_bytes(page_size, idx_dim);
 }
@@ -319,7 +339,6 @@ qsa_status qsa_compress_append(const qsa_cache *cache, int32_t B, const int32_t 
   if (B == 0 || max_new_per_req == 0) return QSA_OK;
   if (B > cache->ring_rows || B > 65535) return QSA_ERR_INVALID_ARG;
   if (!pos0 || !cu_new || !k_new || !cache->kc || !cache->ring) return QSA_ERR_INVALID_ARG;
-  if (cache->page_size % 16 != 0) return QSA_ERR_UNSUPPORTED;  // packed compressed-key pages
   if (!aligned(k_new, 4) || !aligned(cache->kc, 16) || !aligned(cache->ring, 4))
     return QSA_ERR_INVALID_ARG;
   const long long max_blocks = (long long)max_new_per_req / 4 + 2;
@@ -364,7 +383,6 @@ qsa_status index_topk_call(const qsa_cache *cache, int32_t B, const int8_t *q_id
   if (!q_idx || !ctx_lens || !(sel || tokens) || !workspace || !cache->kc) return QSA_ERR_INVALID_ARG;
   if (cache->idx_dim != 32 && cache->idx_dim != 64 && cache->idx_dim != 128)
     return QSA_ERR_UNSUPPORTED;
-  if (cache->page_size % 16 != 0) return QSA_ERR_UNSUPPORTED;  // packed compressed-key pages
   if (!aligned(cache->kc, 16) || !aligned(q_idx, 4) || !aligned(workspace, 16) ||
       (scores && !aligned(scores, 4)) || (tokens && !aligned(tokens, 16)))
     return QSA_ERR_INVALID_ARG;
@@ -384,16 +402,8 @@ qsa_status index_topk_call(const qsa_cache *cache, int32_t B, const int8_t *q_id
   p.T = T;
   p.scores = scores ? scores
                     : reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + kTicketBytes);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int P = cache->page_size;
-  switch (cache->idx_dim) {
-    case 32: return P == 64 ? launch_index_topk<32, 16>(p, s)
-                  : P == 16 ? launch_index_topk<32, 4>(p, s) : launch_index_topk<32, 0>(p, s);
-    case 64: return P == 64 ? launch_index_topk<64, 16>(p, s)
-                  : P == 16 ? launch_index_topk<64, 4>(p, s) : launch_index_topk<64, 0>(p, s);
-    default: return P == 64 ? launch_index_topk<128, 16>(p, s)
-                  : P == 16 ? launch_index_topk<128, 4>(p, s) : launch_index_topk<128, 0>(p, s);
-  }
+  return dispatch_index_topk(p, cache->idx_dim, cache->page_size,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -510,6 +520,12 @@ qsa_status sparse_decode_call(const qsa_cache *cache, int32_t B, int32_t T, int3
   p.nch = nch;  // the launch sets nch and chunk for its kernel
   p.chunk = qsa::dec::kMinChunkBlocks;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the header (work counters, split tickets) starts at zero in every call,
+  // whatever the workspace held
+  const int header_ints = qsa::dec::kCounterInts + B * Hkv * num_splits;
+  st = launch(true, qsa::dec::decode_header_reset_kernel, dim3(1), dim3(1024), 0, s, p.counters,
+              header_ints);
+  if (st != QSA_OK) return st;
   st = (D == 64) ? dispatch_decode_d<64>(p, cache->kv_dtype, s)
                  : dispatch_decode_d<128>(p, cache->kv_dtype, s);
   // the merge kernel, one warp per output row, right behind the decode
@@ -642,7 +658,6 @@ qsa_status qsa_index_topk_noalloc(const qsa_cache *cache, int32_t B, const int8_
   if (!q_idx || !ctx_lens || !sel || !cache->kc) return QSA_ERR_INVALID_ARG;
   if (cache->idx_dim != 32 && cache->idx_dim != 64 && cache->idx_dim != 128)
     return QSA_ERR_UNSUPPORTED;
-  if (cache->page_size % 16 != 0) return QSA_ERR_UNSUPPORTED;  // packed compressed-key pages
   if (!aligned(cache->kc, 16) || !aligned(q_idx, 4)) return QSA_ERR_INVALID_ARG;
   int32_t *scores = noalloc_scores_ptr();
   if (!scores) return QSA_ERR_CUDA;
@@ -657,16 +672,8 @@ qsa_status qsa_index_topk_noalloc(const qsa_cache *cache, int32_t B, const int8_
   p.topk = topk;
   p.sel = sel;
   p.scores = scores;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int P = cache->page_size;
-  switch (cache->idx_dim) {
-    case 32: return P == 64 ? launch_index_topk<32, 16>(p, s)
-                  : P == 16 ? launch_index_topk<32, 4>(p, s) : launch_index_topk<32, 0>(p, s);
-    case 64: return P == 64 ? launch_index_topk<64, 16>(p, s)
-                  : P == 16 ? launch_index_topk<64, 4>(p, s) : launch_index_topk<64, 0>(p, s);
-    default: return P == 64 ? launch_index_topk<128, 16>(p, s)
-                  : P == 16 ? launch_index_topk<128, 4>(p, s) : launch_index_topk<128, 0>(p, s);
-  }
+  return dispatch_index_topk(p, cache->idx_dim, cache->page_size,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -53,14 +53,23 @@ struct Params {
   float *lse_part;  // [S, B, T, Hq]
   float *ws_o;      // [B, Hkv, nch, M, D]
   float *ws_lse;    // [B, Hkv, nch, M]
-  int32_t *tickets;  // [B, Hkv, S]
-  int32_t *counters; // work counters of the persistent kernel (zero between calls)
+  int32_t *tickets;  // [B, Hkv, S], zeroed by the call's reset kernel
+  int32_t *counters; // work counters of the persistent kernels, zeroed likewise
   int nch;           // chunk slots per (r, g)
   int chunk;         // target micro-blocks per chunk, kMinChunkBlocks..kChunkBlocks
   // splits computed: [s_lo, s_hi) of S (a decode-context-parallel rank
   // computes its own); o_part / lse_part hold them from index 0
   int s_lo = 0, s_hi = 0;
 };
+
+// First kernel of every decode call: zeroes the workspace header (the work
+// counters and the split tickets), so the caller's workspace may hold
+// anything.  It goes on the stream right before the decode kernel, both with
+// programmatic launch: the decode's CTAs become resident while this runs.
+__global__ void __launch_bounds__(1024) decode_header_reset_kernel(int32_t *hdr, int n) {
+  pdl_open();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) hdr[i] = 0;
+}
 
 // Per-CTA plan, computed by warp 0.
 struct Plan {
@@ -235,8 +244,7 @@ __device__ void finish_chunk(const Params &p, const Plan &pl, int r, int g, cons
   int32_t *ticket = p.tickets + ((long long)r * Hkv + g) * p.S + s;
   if (threadIdx.x == 0) {
     const int t = atomicAdd(ticket, 1);
-    *flag = (t == pl.nchunks_split - 1);
-    if (*flag) *ticket = 0;  // all chunks of the split have reported
+    *flag = (t == pl.nchunks_split - 1);  // all chunks of the split have reported
   }
   __syncthreads();
   if (!*flag) return;

@@ -353,7 +353,6 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
       int32_t *ticket = p.tickets + ((long long)r * Hkv + g) * p.S + s_idx;
       const int t = atomicAdd(ticket, 1);
       const int is_last = (t == pl.nchunks_split - 1);
-      if (is_last) *ticket = 0;
       sm.last[grp] = is_last;
     }
     gsync();
@@ -394,13 +393,6 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_group_kernel(Params 
       *reinterpret_cast<float4 *>(p.o_part + out_row(p, s_idx, r, g, m) * D + d) =
           make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
       if (d == 0) p.lse_part[out_row(p, s_idx, r, g, m)] = den > 0.f ? mx + __logf(den) : -INFINITY;
-    }
-  }
-  // every group reports once; the last one resets the work counters
-  if (tig == 0) {
-    if (atomicAdd(&p.counters[1], 1) == ngroups - 1) {
-      atomicExch(&p.counters[0], 0);
-      atomicExch(&p.counters[1], 0);
     }
   }
 }

@@ -21,7 +21,7 @@ namespace qsa {
 namespace dec {
 
 constexpr int kTokW = 16;         // tokens per stage
-constexpr int kCounterInts = 64;  // workspace header: [0] next item, [1] finished warps
+constexpr int kCounterInts = 64;  // workspace header: [0] next item (then the split tickets)
 
 // Shared-memory layout of one worker warp: a ring of NS 16-token K/V stages
 // and the chunk's token metadata.
@@ -521,7 +521,6 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p
       int32_t *ticket = p.tickets + ((long long)r * Hkv + g) * p.S + s_idx;
       const int t = atomicAdd(ticket, 1);
       last = (t == pl.nchunks_split - 1);
-      if (last) *ticket = 0;
     }
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) continue;
@@ -564,13 +563,6 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_warp_kernel(Params p
       if (d == 0) p.lse_part[out_row(p, s_idx, r, g, m)] = den > 0.f ? mx + __logf(den) : -INFINITY;
     }
     __syncwarp();
-  }
-  // every warp reports once; the last one resets the work counters
-  if (lane == 0) {
-    if (atomicAdd(&p.counters[1], 1) == nwarps - 1) {
-      atomicExch(&p.counters[0], 0);
-      atomicExch(&p.counters[1], 0);
-    }
   }
 }
 

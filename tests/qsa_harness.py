@@ -219,3 +219,54 @@ def check_properties(batch: QSABatch, step: QSADecodeStep) -> None:
             assert set(pl) <= set(sel[r].tolist()), f"planted r={r}"
     o = step.o.cpu()
     assert bool(torch.isfinite(o).all()) and bool(torch.isfinite(step.lse.cpu()).all())
+
+
+def check_index_every_request(batch: QSABatch, sel: torch.Tensor, scores: torch.Tensor | None,
+                              topk: int | None = None, workers: int = 16) -> int:
+    """Bit-exact comparison of the selection rows (and, when given, the
+    scores) of EVERY request with the oracle's indexer path, run request by
+    request in a pool of spawn worker processes.  The raw keys go to the
+    workers one request at a time, with a bounded number in flight, so host
+    memory stays bounded at any batch size.  Returns the requests checked."""
+    import oracle_index
+    w = batch.w
+    topk = w.topk if topk is None else topk
+    sel_h = sel.cpu().numpy()
+    sc_dev = scores
+    pending = {}
+    checked = 0
+
+    def settle(fut, r):
+        nonlocal checked
+        want_sc, want_sel = fut.result()
+        assert np.array_equal(sel_h[r], want_sel), f"selection mismatch r={r}"
+        if sc_dev is not None:
+            got = sc_dev[r, :want_sc.shape[0]].cpu().numpy().astype(np.int64)
+            assert np.array_equal(got, want_sc), f"score mismatch r={r}"
+        checked += 1
+
+    n_workers = oracle_index.pool_size(workers)
+    with oracle_index.pool(n_workers) as ex:
+        limit = 2 * n_workers
+        for r in range(w.batch):
+            a, e = int(batch.cu_ctx_host[r]), int(batch.cu_ctx_host[r + 1])
+            k = batch.k_idx[a:e].cpu().numpy()
+            q = batch.q_idx[r].cpu().numpy()
+            pending[ex.submit(oracle_index.index_request, k, q, w.T, topk)] = r
+            if len(pending) >= limit:
+                fut = next(iter(pending))
+                settle(fut, pending.pop(fut))
+        for fut, r in list(pending.items()):
+            settle(fut, r)
+    return checked
+
+
+def sample_requests(L: torch.Tensor, k: int = 16) -> list[int]:
+    """k requests spread over the context-length order (shortest and longest
+    included)."""
+    order = torch.argsort(L).tolist()
+    n = len(order)
+    if n <= k:
+        return sorted(order)
+    pick = {order[round(i * (n - 1) / (k - 1))] for i in range(k)}
+    return sorted(pick)

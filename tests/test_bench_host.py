@@ -39,16 +39,21 @@ def test_algorithmic_bytes_fp8_scales_and_mtp_tail():
 
 
 def test_traffic_record_checks_the_kernel_source(tmp_path, monkeypatch):
+    """The record's traffic is reported only for the kernel source it was
+    captured from (checked on a copy of the record pointed at a file of
+    known contents)."""
+    import hashlib
     rec = json.load(open(os.path.join(bench.ROOT, "profiles", "roofline_traffic.json")))
-    got = bench.index_topk_traffic(128)
-    assert got == rec["dram_bytes_per_request"] * 128
-    # a copy of the tree whose kernel source differs: no traffic figure
-    os.makedirs(tmp_path / "profiles")
-    shutil.copy(os.path.join(bench.ROOT, "profiles", "roofline_traffic.json"), tmp_path / "profiles")
     src = tmp_path / rec["source"]
     os.makedirs(src.parent)
-    src.write_text(open(os.path.join(bench.ROOT, rec["source"])).read() + "\n// changed\n")
+    src.write_text("// kernel source\n")
+    rec["source_sha256_prefix"] = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    os.makedirs(tmp_path / "profiles")
+    with open(tmp_path / "profiles" / "roofline_traffic.json", "w") as f:
+        json.dump(rec, f)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.index_topk_traffic(128) == rec["dram_bytes_per_request"] * 128
+    src.write_text("// kernel source\n// changed\n")   # the source moved on: no figure
     assert bench.index_topk_traffic(128) is None
 
 
@@ -65,3 +70,8 @@ def test_l2_statement():
     big = bench.workload_config(WORKLOADS["b128_256k"], 2, 1)["l2"]
     small = bench.workload_config(WORKLOADS["tiny"], 1, 1)["l2"]
     assert big.startswith("inputs larger than L2") and small.startswith("inputs smaller than L2")
+
+
+def test_parallel_oracle_timing_counts_every_core():
+    res = bench.time_oracle_parallel(WORKLOADS["tiny"], 1, 1, 2)
+    assert res["cores"] == 2 and res["queries"] == 2 and res["value"] > 0

@@ -233,21 +233,18 @@ def test_host_validation_rejects_bad_arguments():
 
 # ------------------------------------------------------------ full sizes --
 
-def _sample(L: torch.Tensor, k: int = 3) -> list[int]:
-    order = torch.argsort(L)
-    pick = {int(order[0]), int(order[len(order) // 2]), int(order[-1])}
-    return sorted(pick)[:k]
-
-
 @pytest.mark.parametrize("name,S", [("b32_32k", 2), ("b128_256k", 2), ("mtp_verify", 2),
                                     ("mixed_fp8", 4)])
-def test_full_size_sampled(name, S):
+def test_full_size(name, S):
     """Full-size workloads in the launch configuration of the benchmark:
-    element-wise parity on sampled requests, properties on every request."""
+    scores and selected blocks bit-exact against the oracle on EVERY
+    request; compressed keys, ring and attention element-wise on 16 requests
+    spread over the context lengths; properties on every request."""
     b = make_batch(WORKLOADS[name], "cuda")
     step, cache = H.run_gpu(b, S)
     H.check_properties(b, step)
-    for r in _sample(b.ctx_lens_host):
+    assert H.check_index_every_request(b, step.sel, step.scores) == b.w.batch
+    for r in H.sample_requests(b.ctx_lens_host, 16):
         H.check_request(b, step, cache, r, S)
     del step, cache, b
 
@@ -266,3 +263,26 @@ def test_full_size_256k_split_invariance():
             assert torch.equal(step.sel, ref_sel)
             assert float((step.o - ref_o).abs().max()) < 1e-4
             H.check_request(b, step, cache, 127, S, check_kc=False)
+
+
+@pytest.mark.parametrize("name,lens,S", [("b32_32k", [9000, 12345, 4099], 2),
+                                         ("mtp_verify", [16384 + 3, 9001], 2),
+                                         ("mixed_fp8", [4096, 30007], 4),
+                                         ("tiny", None, 1)])
+def test_decode_workspace_of_any_contents(name, lens, S):
+    """The decode zeroes its workspace header (work counter, split tickets)
+    itself: a workspace full of garbage gives the same bits as a zeroed one,
+    call after call."""
+    from sparse_attention_decode_compress_b200 import api
+    b = make_batch(WORKLOADS[name], "cuda", ctx_lens=lens, seed=19)
+    step, cache = H.run_gpu(b, S, keep_scores=False)
+    for fill in (0xFF, 0x7F, 0x01):
+        step.ws_dec.fill_(fill)
+        o_part = torch.empty_like(step.o_part)
+        lse_part = torch.empty_like(step.lse_part)
+        for _ in range(2):
+            api.qsa_sparse_decode(cache, b.q, b.ctx_lens, step.sel, step.sm_scale, S, o_part,
+                                  lse_part, step.ws_dec)
+            st, flags = api.qsa_get_device_error()
+            assert st == 0, (fill, st, flags)
+            assert torch.equal(o_part, step.o_part) and torch.equal(lse_part, step.lse_part)

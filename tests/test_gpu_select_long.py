@@ -65,3 +65,24 @@ def test_all_keys_equal_long_requests():
 def test_small_topk(topk):
     w = replace(WORKLOADS["b32_32k"], planted=4, topk=topk)
     _check(make_batch(w, "cuda", ctx_lens=[32768, 20001, 77777], seed=24 + topk), 2)
+
+
+# Requests of more than 262,144 micro-blocks keep their kept blocks in a list
+# instead of the shared bitmap, and a topk above 1024 writes that list out
+# with a bitonic sort: one request of 1,048,580 tokens (262,145 blocks)
+# takes both branches.
+@pytest.mark.parametrize("topk", [512, 2048])
+def test_requests_beyond_the_bitmap_use_the_kept_list(topk):
+    w = replace(WORKLOADS["b128_256k"], planted=8, topk=topk)
+    _check(make_batch(w, "cuda", ctx_lens=[1048580, 70001], seed=31), 2)
+
+
+def test_beyond_the_bitmap_with_every_score_tied():
+    # the exact fallback, then the kept list and its bitonic sort
+    w = replace(WORKLOADS["b128_256k"], planted=0, topk=2048)
+    b = make_batch(w, "cuda", ctx_lens=[1048580, 9000], seed=32)
+    b.k_idx.fill_(5)
+    step, cache = H.run_gpu(b, 2)
+    assert step.sel[0].cpu().tolist() == list(range(2048))
+    for r in range(b.w.batch):
+        H.check_request(b, step, cache, r, 2)

@@ -23,7 +23,8 @@ def _pack(vals: np.ndarray, P: int, d: int, page_bytes: int) -> np.ndarray:
     return out
 
 
-@pytest.mark.parametrize("P,d", [(64, 128), (16, 32), (64, 64), (32, 32), (16, 128)])
+@pytest.mark.parametrize("P,d", [(64, 128), (16, 32), (64, 64), (32, 32), (16, 128), (4, 128),
+                                 (8, 32), (12, 64), (20, 128), (4, 32)])
 def test_page_bytes(P, d):
     lib = _lib.load()
     R = P // 4
@@ -33,13 +34,13 @@ def test_page_bytes(P, d):
 
 def test_page_bytes_rejects_bad_geometry():
     lib = _lib.load()
-    assert lib.qsa_kc_page_bytes(6, 128) == 0
-    assert lib.qsa_kc_page_bytes(8, 128) == 0   # pages hold whole 4-row runs: P % 16 == 0
+    assert lib.qsa_kc_page_bytes(6, 128) == 0   # pages hold whole micro-blocks: P % 4 == 0
+    assert lib.qsa_kc_page_bytes(2, 32) == 0
     assert lib.qsa_kc_page_bytes(64, 48) == 0
     assert lib.qsa_kc_page_bytes(0, 128) == 0
 
 
-@pytest.mark.parametrize("P,d", [(64, 128), (16, 32), (32, 64)])
+@pytest.mark.parametrize("P,d", [(64, 128), (16, 32), (32, 64), (4, 128), (12, 32), (20, 64)])
 def test_harness_reader_round_trip(P, d):
     lib = _lib.load()
     rng = np.random.default_rng(P * d)
@@ -58,8 +59,11 @@ def test_cache_allocation_uses_the_packed_page():
     c = QSACache.allocate(k, k.clone(), bt, idx_dim=128, ring_rows=1)
     assert c.kc.dtype == torch.uint8 and tuple(c.kc.shape) == (5, 16 * 128 + 16 * 32)
     k8 = torch.zeros((5, 8, 2, 128), dtype=torch.bfloat16)
+    c8 = QSACache.allocate(k8, k8.clone(), bt, idx_dim=128, ring_rows=1)
+    assert tuple(c8.kc.shape) == (5, 2 * 128 + 64)
+    k6 = torch.zeros((5, 6, 2, 128), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="unsupported compressed-key geometry"):
-        QSACache.allocate(k8, k8.clone(), bt, idx_dim=128, ring_rows=1)
+        QSACache.allocate(k6, k6.clone(), bt, idx_dim=128, ring_rows=1)
     # an int16-shaped cache is rejected before any pointer is taken
     bad = QSACache(k, k.clone(), torch.zeros((5, 4096), dtype=torch.uint8), c.ring, bt)
     with pytest.raises(ValueError, match="qsa_kc_page_bytes"):
