@@ -336,6 +336,56 @@ qsa_status qsa_lse_merge(int32_t num_splits, int64_t rows, int32_t D, const floa
                          const float *lse_part, float *o, float *lse, qsa_stream_t stream);
 
 /*
+ * Normalised-pooling indexer variant: float compressed keys and scores.
+ *
+ * Passage: PR #53896 report, QSAIndexer.forward excerpt under 关键源码片段
+ * (raw token keys are pooled by the compress ratio and normalised before
+ * they enter the compressed-key cache) and 实现拆解 (an RMS norm of the
+ * indexer, apply_qsa_rmsnorm).  Reading: pooling = mean of the tokens present
+ * in the micro-block; normalisation = RMS normalisation,
+ *     k_c[b] = m_b / sqrt(mean_j m_b[j]^2 + eps) * (1 + w),  m_b = block mean,
+ * w an optional per-dim weight; score[r][b] = q_r . k_c[b] in float; the
+ * selection rule is qsa_index_topk's (highest score first, ties: lower block
+ * index; ascending; -1 padded).
+ *
+ * Storage (separate from the integer indexer's caches; same block table):
+ *   kcn   [num_pages, qsa_kcn_page_bytes(P, d)] bytes: page = [P/4 rows][d]
+ *         float16 compressed keys, 16-byte aligned
+ *   ring  [ring_rows, 4, d] bfloat16: slot p % 4 of row r holds request r's
+ *         raw key at position p, 16-byte aligned
+ * Numerics: sums, the mean square and the dot products in float32; k_c is
+ * rounded to float16 (relative error <= 2^-11), so a score is within
+ * 2^-10 * |q|_2 * sqrt(d) * max_j |1 + w_j| of the exact one, and blocks whose
+ * scores are that close to the top-k threshold may be ordered either way.
+ *
+ * qsa_kcn_page_bytes: (P/4) * d * 2, or 0 for page_size not a positive
+ * multiple of 4 or idx_dim not 32, 64 or 128.
+ *
+ * qsa_compress_append_norm: as qsa_compress_append (pos0, cu_new,
+ * max_new_per_req, ring_rows and the append order are the same), with
+ *   k_new        [N, d] bfloat16 raw keys, 16-byte aligned
+ *   norm_weight  [d] float32 w, or NULL for none
+ *   eps          > 0 (1e-6 in the tests)
+ * Errors: QSA_ERR_INVALID_ARG for null or misaligned pointers, B out of
+ * range, eps <= 0; QSA_ERR_UNSUPPORTED for an unsupported idx_dim.
+ *
+ * qsa_index_topk_norm: as qsa_index_topk (ctx_lens, n_sel, max_blocks,
+ * topk, sel, workspace of qsa_index_topk_workspace_bytes), with
+ *   q_idx   [B, d] bfloat16 indexer query, 16-byte aligned
+ *   scores  [B, max_blocks] float32 output of every score, or NULL
+ * Two kernels: a scan of the float16 keys and the selection on float keys.
+ */
+size_t qsa_kcn_page_bytes(int32_t page_size, int32_t idx_dim);
+qsa_status qsa_compress_append_norm(const qsa_cache *cache, void *kcn, void *ring,
+                                    const float *norm_weight, float eps, int32_t B,
+                                    const int32_t *pos0, const int32_t *cu_new, const void *k_new,
+                                    int32_t max_new_per_req, qsa_stream_t stream);
+qsa_status qsa_index_topk_norm(const qsa_cache *cache, const void *kcn, int32_t B,
+                               const void *q_idx, const int32_t *ctx_lens, const int32_t *n_sel,
+                               int32_t max_blocks, int32_t topk, int32_t *sel, float *scores,
+                               void *workspace, size_t workspace_bytes, qsa_stream_t stream);
+
+/*
  * qsa_index_topk_noalloc — qsa_index_topk without a caller workspace.
  *
  * The source pages have no counterpart to this entry point; it exists for

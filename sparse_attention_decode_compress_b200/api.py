@@ -300,6 +300,83 @@ def qsa_lse_merge(o_part: torch.Tensor, lse_part: torch.Tensor, o: torch.Tensor,
                              _stream(stream)), "qsa_lse_merge")
 
 
+def qsa_kcn_page_bytes(page_size: int, idx_dim: int) -> int:
+    return int(_lib.load().qsa_kcn_page_bytes(page_size, idx_dim))
+
+
+def allocate_norm_caches(cache: QSACache, ring_rows: int) -> tuple[torch.Tensor, torch.Tensor]:
+    """Side caches of the normalised-pooling indexer, in the cache group of
+    `cache` (its block table names their pages): float16 compressed keys
+    [num_pages, P/4, d] and the bfloat16 raw-key ring [ring_rows, 4, d]."""
+    num_pages, P = cache.k_cache.shape[0], cache.k_cache.shape[1]
+    d = cache.ring.shape[-1]
+    if qsa_kcn_page_bytes(P, d) == 0:
+        raise ValueError(f"unsupported compressed-key geometry: page_size {P}, idx_dim {d}")
+    dev = cache.k_cache.device
+    kcn = torch.zeros((num_pages, P // 4, d), dtype=torch.float16, device=dev)
+    ring = torch.zeros((ring_rows, 4, d), dtype=torch.bfloat16, device=dev)
+    return kcn, ring
+
+
+def _check_norm_caches(cache: QSACache, kcn: torch.Tensor, ring: torch.Tensor):
+    num_pages, P = cache.k_cache.shape[0], cache.k_cache.shape[1]
+    d = cache.ring.shape[-1]
+    _need(kcn, torch.float16, "kcn")
+    _need(ring, torch.bfloat16, "ring")
+    if tuple(kcn.shape) != (num_pages, P // 4, d) or ring.dim() != 3 or ring.shape[1:] != (4, d):
+        raise ValueError("kcn must be [num_pages, P/4, d] float16 and ring [rows, 4, d] bfloat16")
+
+
+def qsa_compress_append_norm(cache: QSACache, kcn: torch.Tensor, ring: torch.Tensor,
+                             norm_weight: torch.Tensor | None, eps: float, pos0: torch.Tensor,
+                             cu_new: torch.Tensor, k_new: torch.Tensor, max_new_per_req: int,
+                             stream=None) -> None:
+    """Normalised-pooling compress-append: bfloat16 raw keys k_new [N, d]
+    into the ring and the float16 compressed-key pages."""
+    _check_norm_caches(cache, kcn, ring)
+    _need(pos0, torch.int32, "pos0")
+    _need(cu_new, torch.int32, "cu_new")
+    _need(k_new, torch.bfloat16, "k_new")
+    if norm_weight is not None:
+        _need(norm_weight, torch.float32, "norm_weight")
+    B = pos0.shape[0]
+    if cu_new.shape[0] != B + 1:
+        raise ValueError("cu_new must have B+1 entries")
+    s = cache.struct()
+    s.ring_rows = ring.shape[0]
+    _check(_lib.load().qsa_compress_append_norm(ctypes.byref(s), _ptr(kcn), _ptr(ring),
+                                                _ptr(norm_weight), float(eps), B, _ptr(pos0),
+                                                _ptr(cu_new), _ptr(k_new), int(max_new_per_req),
+                                                _stream(stream)), "qsa_compress_append_norm")
+
+
+def qsa_index_topk_norm(cache: QSACache, kcn: torch.Tensor, q_idx: torch.Tensor,
+                        ctx_lens: torch.Tensor, n_sel: torch.Tensor | None, max_blocks: int,
+                        topk: int, sel: torch.Tensor, scores: torch.Tensor | None,
+                        workspace: torch.Tensor, stream=None) -> None:
+    """Float scores of the normalised compressed keys against the bfloat16
+    indexer query q_idx [B, d], and the top-k selection on them."""
+    _need(kcn, torch.float16, "kcn")
+    _need(q_idx, torch.bfloat16, "q_idx")
+    _need(ctx_lens, torch.int32, "ctx_lens")
+    _need(sel, torch.int32, "sel")
+    B = q_idx.shape[0]
+    if sel.shape != (B, topk):
+        raise ValueError("sel must be [B, topk]")
+    if n_sel is not None:
+        _need(n_sel, torch.int32, "n_sel")
+    if scores is not None:
+        _need(scores, torch.float32, "scores")
+        if scores.shape != (B, max_blocks):
+            raise ValueError("scores must be [B, max_blocks]")
+    s = cache.struct()
+    _check(_lib.load().qsa_index_topk_norm(ctypes.byref(s), _ptr(kcn), B, _ptr(q_idx),
+                                           _ptr(ctx_lens), _ptr(n_sel), int(max_blocks), int(topk),
+                                           _ptr(sel), _ptr(scores), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(),
+                                           _stream(stream)), "qsa_index_topk_norm")
+
+
 class QSASession:
     """Decode steps from host buffers to host buffers (qsa_session_*): the
     library owns the device buffers and overlaps each step's uploads and

@@ -30,11 +30,12 @@
 namespace qsa {
 namespace topk {
 
-// Scores are ordered through 25-bit keys, score + 2^24: |score| <= 2^23 for
-// d <= 128 and int8 inputs.  The first digit is key bits [24:12] (8192 bins
-// of 4096 score units); the exact fallback resolves bits [11:6] and [5:0].
+// Integer scores are ordered through 25-bit keys, score + 2^24: |score| <=
+// 2^23 for d <= 128 and int8 inputs.  The first digit is key bits [24:12]
+// (8192 bins of 4096 score units); the exact fallback resolves bits [11:6]
+// and [5:0].  Float scores use 32-bit keys the same way (IntKeys /
+// FloatKeys below).
 constexpr int kScoreBias = 1 << 24;
-constexpr int kDigit1Shift = 12;
 constexpr int kHistBins = 1 << 13;
 constexpr int kFbDigitBits = 6;
 constexpr int kCandCap = 2048;   // threshold-bin candidates kept in shared memory
@@ -76,6 +77,28 @@ __device__ __forceinline__ uint32_t score_key(int s) {
   s = max(min(s, kScoreBias - 1), -kScoreBias);
   return (uint32_t)(s + kScoreBias);
 }
+
+// How the selection orders the 32-bit words of a score row: an unsigned key
+// of kBits bits, larger for a better score (ties: lower block index wins).
+// The first digit is the key's top 13 bits; the exact fallback resolves the
+// bits below in digits of at most kFbDigitBits.
+struct IntKeys {  // int32 scores of the integer indexer
+  static constexpr int kBits = 25;
+  __device__ __forceinline__ static uint32_t key(int s) { return score_key(s); }
+  __device__ __forceinline__ static uint32_t quad_max(int4 v) {
+    return score_key(max(max(v.x, v.y), max(v.z, v.w)));
+  }
+};
+struct FloatKeys {  // float32 scores (their bits) of the normalised indexer
+  static constexpr int kBits = 32;
+  __device__ __forceinline__ static uint32_t key(int bits) {
+    const uint32_t u = (uint32_t)bits;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  }
+  __device__ __forceinline__ static uint32_t quad_max(int4 v) {
+    return max(max(key(v.x), key(v.y)), max(key(v.z), key(v.w)));
+  }
+};
 
 // ------------------------------------------------------------ selection --
 // One CTA of kSelThreads threads per request.  The request's scores (written
@@ -320,24 +343,26 @@ __device__ void find_rank_bin_desc(const int *hist, int rank, SelSmem &sm, int t
 // radix passes over the score row establish the exact threshold key, then
 // (on a tie at the threshold) the largest kept index among the tied blocks,
 // then the kept set is gathered.
+template <typename KT>
 __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, int tid) {
   int *hist = sm.hist;
-  constexpr int kFbBins = 1 << kFbDigitBits;
+  constexpr int kShift1 = KT::kBits - 13;
   uint32_t prefix = (uint32_t)sm.bin;  // key >> shift
   int above = sm.above;
-  int shift = kDigit1Shift;
-  for (int pass = 0; pass < 2; ++pass) {
-    const int nshift = shift - kFbDigitBits;
+  for (int shift = kShift1; shift > 0;) {
+    const int nbits = min(kFbDigitBits, shift);
+    const int nshift = shift - nbits;
+    const int nbins = 1 << nbits;
     for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
     __syncthreads();
     for_each_score(sc, n, tid, [&](int, int s) {
-      const uint32_t k = score_key(s);
-      if ((k >> shift) == prefix) atomicAdd(&hist[(k >> nshift) & (kFbBins - 1)], 1);
+      const uint32_t k = KT::key(s);
+      if ((k >> shift) == prefix) atomicAdd(&hist[(k >> nshift) & (nbins - 1)], 1);
     });
     __syncthreads();
     if (tid == 0) {
       int cum = above;
-      for (int b = kFbBins - 1; b >= 0; --b) {
+      for (int b = nbins - 1; b >= 0; --b) {
         if (cum + hist[b] >= K) {
           sm.fb_key = b;
           sm.fb_above = cum;
@@ -347,7 +372,7 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
       }
     }
     __syncthreads();
-    prefix = (prefix << kFbDigitBits) | (uint32_t)sm.fb_key;
+    prefix = (prefix << nbits) | (uint32_t)sm.fb_key;
     above = sm.fb_above;
     shift = nshift;
   }
@@ -356,7 +381,7 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
   if (tid == 0) sm.ncand = 0;
   __syncthreads();
   int myties = 0;
-  for_each_score(sc, n, tid, [&](int, int s) { myties += (score_key(s) == tkey); });
+  for_each_score(sc, n, tid, [&](int, int s) { myties += (KT::key(s) == tkey); });
   atomicAdd(&sm.ncand, myties);
   __syncthreads();
   int idx_limit = 0x7fffffff;
@@ -369,7 +394,7 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
       for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
       __syncthreads();
       for_each_score(sc, n, tid, [&](int i, int s) {
-        if (score_key(s) == tkey && ((uint32_t)i >> (sh + 8)) == ipre)
+        if (KT::key(s) == tkey && ((uint32_t)i >> (sh + 8)) == ipre)
           atomicAdd(&hist[((uint32_t)i >> sh) & 255], 1);
       });
       __syncthreads();
@@ -394,7 +419,7 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
   if (tid == 0) sm.nkeep = 0;
   __syncthreads();
   for_each_score(sc, n, tid, [&](int i, int s) {
-    const uint32_t k = score_key(s);
+    const uint32_t k = KT::key(s);
     if (k > tkey || (k == tkey && i <= idx_limit)) {
       const int slot = atomicAdd(&sm.nkeep, 1);
       if (slot < kMaxTopk) keep[slot] = i;
@@ -427,18 +452,20 @@ __device__ void write_ascending(int *keep, int K, int32_t *out, int32_t *tok, in
 // first digit, then a pass that keeps the blocks above the threshold bin
 // (bitmap when use_bits, else the list in sm.hist) and gathers the bin's
 // blocks.
+template <typename KT>
 __device__ void select_passes(const int32_t *sc, int n, int K, bool use_bits, SelSmem &sm,
                                int tid) {
+  constexpr int kShift1 = KT::kBits - 13;
   for_each_score(sc, n, tid, [&](int, int sv) {
-    atomicAdd(&sm.hist[score_key(sv) >> kDigit1Shift], 1);
+    atomicAdd(&sm.hist[KT::key(sv) >> kShift1], 1);
   });
   __syncthreads();
   find_rank_bin_desc(sm.hist, K, sm, tid);
   const uint32_t b1 = (uint32_t)sm.bin;
   int *keep = sm.hist;
   auto visit = [&](int i, int sv) {
-    const uint32_t k = score_key(sv);
-    const uint32_t d1 = k >> kDigit1Shift;
+    const uint32_t k = KT::key(sv);
+    const uint32_t d1 = k >> kShift1;
     if (d1 > b1) {
       if (use_bits) {
         atomicOr(&sm.bits[i >> 5], 1u << (i & 31));
@@ -449,18 +476,14 @@ __device__ void select_passes(const int32_t *sc, int n, int K, bool use_bits, Se
     }
     append_cand(d1 == b1, ((unsigned long long)(0xffffffffu - k) << 32) | (uint32_t)i, sm);
   };
-  // a quad whose largest score is below the threshold bin is skipped whole
+  // a quad whose largest key is below the threshold bin is skipped whole
   for_each_flagged_score(
-      sc, n, tid,
-      [&](int4 v) {
-        const int m = max(max(v.x, v.y), max(v.z, v.w));
-        return (score_key(m) >> kDigit1Shift) >= b1;
-      },
-      visit);
+      sc, n, tid, [&](int4 v) { return (KT::quad_max(v) >> kShift1) >= b1; }, visit);
   __syncthreads();
 }
 
 // Selection kernel: grid = B, one request per CTA.
+template <typename KT>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
   pdl_open();
   extern __shared__ uint8_t smem_raw[];
@@ -494,7 +517,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
     sm.ncand = 0;
   }
   __syncthreads();
-  select_passes(sc, n, K, use_bits, sm, tid);
+  select_passes<KT>(sc, n, K, use_bits, sm, tid);
   int *keep = sm.hist;
   const int above = sm.above;
   const int ncand = sm.ncand;
@@ -515,7 +538,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
     }
     __syncthreads();
   } else {
-    select_fallback(sc, n, K, sm, tid);  // the kept list, in sm.hist
+    select_fallback<KT>(sc, n, K, sm, tid);  // the kept list, in sm.hist
     if (use_bits) {
       for (int i = tid; i < nwords; i += kSelThreads) sm.bits[i] = 0u;
       __syncthreads();

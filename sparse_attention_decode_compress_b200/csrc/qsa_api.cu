@@ -13,6 +13,7 @@
 #include "qsa_common.cuh"
 #include "compress_append.cuh"
 #include "index_topk.cuh"
+#include "index_norm.cuh"
 #include "sparse_decode.cuh"
 #include "sparse_decode_warp.cuh"
 #include "sparse_decode_group.cuh"
@@ -138,7 +139,8 @@ qsa_status launch_index_topk(const qsa::topk::Params &p, cudaStream_t stream) {
   const int dev = current_device();
   {
     std::lock_guard<std::mutex> lk(g_mutex);
-    if (prepare_kernel(select_kernel, select_smem(), done_sel) != cudaSuccess) return QSA_ERR_CUDA;
+    if (prepare_kernel(select_kernel<IntKeys>, select_smem(), done_sel) != cudaSuccess)
+      return QSA_ERR_CUDA;
     if (dev >= 0 && dev < kMaxDevices && !blocks_per_sm[dev]) {
       int n = 0;
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kScanThreads, 0) != cudaSuccess)
@@ -150,7 +152,7 @@ qsa_status launch_index_topk(const qsa::topk::Params &p, cudaStream_t stream) {
   const int grid = bps * sm_count(dev);
   qsa_status st = launch(true, kernel, dim3(grid), dim3(kScanThreads), 0, stream, p);
   if (st != QSA_OK) return st;
-  return launch(true, select_kernel, dim3(p.B), dim3(kSelThreads), select_smem(), stream, p);
+  return launch(true, select_kernel<IntKeys>, dim3(p.B), dim3(kSelThreads), select_smem(), stream, p);
 }
 
 // Scan instance for the indexer dim and page geometry: constant page
@@ -603,6 +605,127 @@ qsa_status qsa_get_device_error(qsa_stream_t stream, uint32_t *flags_out) {
   if (flags & qsa::kErrBounds) return QSA_ERR_BOUNDS;
   if (flags & qsa::kErrBadInput) return QSA_ERR_BAD_INPUT;
   return QSA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Normalised-pooling indexer (float compressed keys, float scores).
+// ---------------------------------------------------------------------------
+namespace {
+
+template <int DI>
+qsa_status launch_index_topk_norm(const qsa::norm::ScanParams &sp, cudaStream_t stream) {
+  using namespace qsa::topk;
+  static bool done_sel[kMaxDevices] = {false};
+  static int blocks_per_sm[kMaxDevices] = {0};
+  auto kernel = qsa::norm::index_scan_norm_kernel<DI>;
+  const int dev = current_device();
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (prepare_kernel(select_kernel<FloatKeys>, select_smem(), done_sel) != cudaSuccess)
+      return QSA_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices && !blocks_per_sm[dev]) {
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, qsa::norm::kScanThreads, 0) !=
+          cudaSuccess)
+        return QSA_ERR_CUDA;
+      blocks_per_sm[dev] = n > 0 ? n : 1;
+    }
+  }
+  const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
+  qsa_status st = launch(true, kernel, dim3(bps * sm_count(dev)), dim3(qsa::norm::kScanThreads), 0,
+                         stream, sp);
+  if (st != QSA_OK) return st;
+  return launch(true, select_kernel<FloatKeys>, dim3(sp.p.B), dim3(kSelThreads), select_smem(),
+                stream, sp.p);
+}
+
+bool norm_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+}  // namespace
+
+extern "C" {
+
+size_t qsa_kcn_page_bytes(int32_t page_size, int32_t idx_dim) {
+  if (page_size <= 0 || page_size % 4 != 0 || !norm_dim_ok(idx_dim)) return 0;
+  return (size_t)(page_size / 4) * (size_t)idx_dim * 2;
+}
+
+qsa_status qsa_compress_append_norm(const qsa_cache *cache, void *kcn, void *ring,
+                                    const float *norm_weight, float eps, int32_t B,
+                                    const int32_t *pos0, const int32_t *cu_new, const void *k_new,
+                                    int32_t max_new_per_req, qsa_stream_t stream) {
+  qsa_status st = check_cache(cache);
+  if (st != QSA_OK) return st;
+  if (B < 0 || max_new_per_req < 0 || !(eps > 0.f) || !std::isfinite(eps)) return QSA_ERR_INVALID_ARG;
+  if (!norm_dim_ok(cache->idx_dim)) return QSA_ERR_UNSUPPORTED;
+  if (B == 0 || max_new_per_req == 0) return QSA_OK;
+  if (B > cache->ring_rows || B > 65535) return QSA_ERR_INVALID_ARG;
+  if (!pos0 || !cu_new || !k_new || !kcn || !ring) return QSA_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(kcn, 16) || !aligned(ring, 16) ||
+      (norm_weight && !aligned(norm_weight, 4)))
+    return QSA_ERR_INVALID_ARG;
+  const long long max_blocks = (long long)max_new_per_req / 4 + 2;
+  const long long gx = (max_blocks + qsa::norm::kAppendBlocksPerCta - 1) / qsa::norm::kAppendBlocksPerCta;
+  if (gx > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  qsa::norm::AppendParams a;
+  a.c = to_dev(cache);
+  a.kcn = static_cast<__half *>(kcn);
+  a.ring = static_cast<__nv_bfloat16 *>(ring);
+  a.weight = norm_weight;
+  a.eps = eps;
+  a.B = B;
+  a.pos0 = pos0;
+  a.cu_new = cu_new;
+  a.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+  a.max_new = max_new_per_req;
+  const dim3 grid((unsigned)gx, (unsigned)B), block(qsa::norm::kAppendThreads);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (cache->idx_dim) {
+    case 32: return launch(false, qsa::norm::compress_append_norm_kernel<32>, grid, block, 0, s, a);
+    case 64: return launch(false, qsa::norm::compress_append_norm_kernel<64>, grid, block, 0, s, a);
+    default: return launch(false, qsa::norm::compress_append_norm_kernel<128>, grid, block, 0, s, a);
+  }
+}
+
+qsa_status qsa_index_topk_norm(const qsa_cache *cache, const void *kcn, int32_t B,
+                               const void *q_idx, const int32_t *ctx_lens, const int32_t *n_sel,
+                               int32_t max_blocks, int32_t topk, int32_t *sel, float *scores,
+                               void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
+  qsa_status st = check_cache(cache);
+  if (st != QSA_OK) return st;
+  if (B < 0) return QSA_ERR_INVALID_ARG;
+  if (topk < 1 || topk > qsa::topk::kMaxTopk) return QSA_ERR_INVALID_ARG;
+  if (max_blocks < 1 || max_blocks > (1 << 24)) return QSA_ERR_INVALID_ARG;
+  if (!norm_dim_ok(cache->idx_dim)) return QSA_ERR_UNSUPPORTED;
+  if (B == 0) return QSA_OK;
+  if (B > 0x7fffffff / 2) return QSA_ERR_UNSUPPORTED;
+  if (!kcn || !q_idx || !ctx_lens || !sel || !workspace) return QSA_ERR_INVALID_ARG;
+  if (!aligned(kcn, 16) || !aligned(q_idx, 16) || !aligned(workspace, 16) ||
+      (scores && !aligned(scores, 4)))
+    return QSA_ERR_INVALID_ARG;
+  const size_t need = scores ? kTicketBytes : qsa_index_topk_workspace_bytes(B, max_blocks);
+  if (workspace_bytes < need) return QSA_ERR_INVALID_ARG;
+  qsa::norm::ScanParams sp;
+  sp.p.c = to_dev(cache);
+  sp.p.B = B;
+  sp.p.q_idx = nullptr;
+  sp.p.ctx_lens = ctx_lens;
+  sp.p.n_sel = n_sel;
+  sp.p.max_blocks = max_blocks;
+  sp.p.topk = topk;
+  sp.p.sel = sel;
+  sp.p.scores = scores ? reinterpret_cast<int32_t *>(scores)
+                       : reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + kTicketBytes);
+  sp.kcn = static_cast<const __half *>(kcn);
+  sp.q = static_cast<const __nv_bfloat16 *>(q_idx);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (cache->idx_dim) {
+    case 32: return launch_index_topk_norm<32>(sp, s);
+    case 64: return launch_index_topk_norm<64>(sp, s);
+    default: return launch_index_topk_norm<128>(sp, s);
+  }
 }
 
 }  // extern "C"

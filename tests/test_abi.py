@@ -114,3 +114,30 @@ def test_page_sizes_of_whole_micro_blocks_have_packed_pages():
         assert lib.qsa_kc_page_bytes(P, 128) > 0
     for P in (2, 6, 10, 18):
         assert lib.qsa_kc_page_bytes(P, 128) == 0
+
+
+def test_norm_indexer_rejects_bad_arguments_on_the_host():
+    lib = _lib.load()
+    c = _cache()
+    assert lib.qsa_kcn_page_bytes(64, 128) == 16 * 128 * 2
+    assert lib.qsa_kcn_page_bytes(12, 32) == 3 * 32 * 2
+    assert lib.qsa_kcn_page_bytes(6, 128) == 0 and lib.qsa_kcn_page_bytes(64, 48) == 0
+    # eps must be positive; pointers 16-byte aligned; B within the ring
+    assert lib.qsa_compress_append_norm(ctypes.byref(c), 0x100, 0x100, None, 0.0, 1, 0x100,
+                                        0x100, 0x100, 1, None) == 1
+    assert lib.qsa_compress_append_norm(ctypes.byref(c), 0x108, 0x100, None, 1e-6, 1, 0x100,
+                                        0x100, 0x100, 1, None) == 1
+    assert lib.qsa_compress_append_norm(ctypes.byref(c), 0x100, 0x100, None, 1e-6, 5, 0x100,
+                                        0x100, 0x100, 1, None) == 1
+    c48 = _cache(idx_dim=48)
+    assert lib.qsa_compress_append_norm(ctypes.byref(c48), 0x100, 0x100, None, 1e-6, 1, 0x100,
+                                        0x100, 0x100, 1, None) == 2
+    # topk out of range, workspace too small, misaligned query
+    assert lib.qsa_index_topk_norm(ctypes.byref(c), 0x100, 1, 0x100, 0x100, None, 16, 0, 0x100,
+                                   None, 0x100, 1 << 20, None) == 1
+    assert lib.qsa_index_topk_norm(ctypes.byref(c), 0x100, 1, 0x100, 0x100, None, 16, 8, 0x100,
+                                   None, 0x100, 16, None) == 1
+    assert lib.qsa_index_topk_norm(ctypes.byref(c), 0x100, 1, 0x104, 0x100, None, 16, 8, 0x100,
+                                   None, 0x100, 1 << 20, None) == 1
+    assert lib.qsa_index_topk_norm(ctypes.byref(c), 0x100, 0, None, None, None, 16, 8, None, None,
+                                   None, 0, None) == 0

@@ -246,3 +246,29 @@ def request_pages(batch: QSABatch, r: int) -> torch.Tensor:
     L = int(batch.ctx_lens_host[r])
     n = (L + batch.w.page_size - 1) // batch.w.page_size
     return batch.block_table_host[r, :n].to(torch.int64)
+
+
+def norm_indexer_inputs(batch: QSABatch, seed: int = 0, weight_std: float = 0.0) -> dict:
+    """Inputs of the normalised-pooling indexer variant for `batch`: raw
+    indexer keys k [sum L, d] and queries q [B, d], bfloat16 ~ N(0, 1); the
+    planted spans' keys (if any) equal their request's query; an optional
+    per-dim norm weight w ~ N(0, weight_std^2) (float32 [d], None for 0)."""
+    w = batch.w
+    device = batch.device
+    gen = torch.Generator(device=device).manual_seed(seed + 7)
+    n_tok = int(batch.cu_ctx_host[-1])
+    k = torch.randn((n_tok, w.d_idx), generator=gen, device=device,
+                    dtype=torch.float32).to(torch.bfloat16)
+    q = torch.randn((w.batch, w.d_idx), generator=gen, device=device,
+                    dtype=torch.float32).to(torch.bfloat16)
+    if batch.planted_host is not None:
+        for r in range(w.batch):
+            for b in batch.planted_host[r].tolist():
+                if b >= 0:
+                    a = int(batch.cu_ctx_host[r]) + RATIO * b
+                    k[a:a + RATIO] = q[r]
+    weight = None
+    if weight_std > 0:
+        weight = torch.randn(w.d_idx, generator=gen, device=device,
+                             dtype=torch.float32) * weight_std
+    return dict(k=k, q=q, weight=weight)
