@@ -386,6 +386,61 @@ qsa_status qsa_index_topk_norm(const qsa_cache *cache, const void *kcn, int32_t 
                                void *workspace, size_t workspace_bytes, qsa_stream_t stream);
 
 /*
+ * qsa_sparse_prefill — QSA attention of a prefill chunk: many query tokens
+ * per request, each with its own selection.
+ *
+ * Passage: blog "为什么一篇关于未发布架构的 serving PR 仍然值得你花时间" (a native
+ * sparse-prefill kernel for the QSA path, PR #59010); what it computes is
+ * read from the decode path of the same pages: query token p of a request is
+ * a causal query over [0, p].  Its candidate blocks are 0 .. floor(p/4), the
+ * block holding p summing only its tokens <= p; they are scored against p's
+ * own indexer query, the best `topk` kept (ties: lower block index), and p
+ * attends the kept blocks' tokens up to p:
+ *   sel[i]  = the kept blocks of token i, ascending, -1 padded
+ *   o[i]    = sum_t softmax(sm_scale * q[i] . k_t) v_t,  lse[i] = log sum exp
+ * (GQA: query head h reads kv head h / (Hq/Hkv)).  A token of the first
+ * 2,048 positions keeps every block: dense causal attention.
+ *
+ * Preconditions: the chunk's tokens are the NEWEST cached tokens of each
+ * request: their K/V rows and raw indexer keys were written (K/V into the
+ * paged cache, keys through qsa_compress_append) before this call, so
+ * request r holds ctx_lens[r] tokens and its query tokens sit at positions
+ * ctx_lens[r] - n_r .. ctx_lens[r] - 1 (n_r = cu_q[r+1] - cu_q[r]).
+ *
+ *   B, n_tokens    requests, and query tokens in all (= cu_q[B])
+ *   max_q_per_req  host bound of n_r (sizes the launch)
+ *   cu_q     [B+1] int32 row offsets of each request's query tokens
+ *   ctx_lens [B] int32 cached tokens of each request (>= n_r)
+ *   q_idx    [n_tokens, d] int8 indexer queries, 16-byte aligned
+ *   k_chunk  [n_tokens, d] int8 raw indexer keys of the query tokens (as
+ *            appended), 4-byte aligned
+ *   q        [n_tokens, Hq, D] of q_dtype (as qsa_sparse_decode)
+ *   max_blocks  host bound of ceil(ctx_lens[r] / 4) (score row stride)
+ *   topk     1 .. 4096
+ *   sel      [n_tokens, topk] int32 output
+ *   o        [n_tokens, Hq, D] float32 output, 16-byte aligned
+ *   lse      [n_tokens, Hq] float32 output
+ *   workspace >= qsa_sparse_prefill_workspace_bytes(n_tokens, max_blocks,
+ *            Hq, Hkv, D, topk) bytes, 256-byte aligned, any contents
+ * Kernels: a tensor-core scan (tcgen05.mma kind::i8, int32 accumulators in
+ * tensor memory) of every token's indexer query against its prefix's
+ * compressed keys, a per-token fix-up of the block holding the token, the
+ * selection of qsa_index_topk per token, and the decode kernels of
+ * qsa_sparse_decode with one split per token.
+ * Errors: QSA_ERR_INVALID_ARG for null / misaligned pointers or sizes out of
+ * range; QSA_ERR_UNSUPPORTED for n_tokens or B above 65535 or an
+ * unsupported idx_dim / head shape; device problems as qsa_sparse_decode.
+ */
+size_t qsa_sparse_prefill_workspace_bytes(int32_t n_tokens, int32_t max_blocks, int32_t Hq,
+                                          int32_t Hkv, int32_t D, int32_t topk);
+qsa_status qsa_sparse_prefill(const qsa_cache *cache, int32_t B, int32_t n_tokens,
+                              int32_t max_q_per_req, const int32_t *cu_q, const int32_t *ctx_lens,
+                              const int8_t *q_idx, const int8_t *k_chunk, const void *q,
+                              int32_t q_dtype, int32_t Hq, int32_t max_blocks, int32_t topk,
+                              float sm_scale, int32_t *sel, float *o, float *lse, void *workspace,
+                              size_t workspace_bytes, qsa_stream_t stream);
+
+/*
  * qsa_index_topk_noalloc — qsa_index_topk without a caller workspace.
  *
  * The source pages have no counterpart to this entry point; it exists for

@@ -62,6 +62,11 @@ SIGNATURES = {
     "qsa_index_topk_norm": (c_int32, [ctypes.POINTER(QsaCacheStruct), c_void_p, c_int32, c_void_p,
                                       c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p,
                                       c_void_p, c_size_t, c_void_p]),
+    "qsa_sparse_prefill_workspace_bytes": (c_size_t, [c_int32] * 6),
+    "qsa_sparse_prefill": (c_int32, [ctypes.POINTER(QsaCacheStruct), c_int32, c_int32, c_int32,
+                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int32,
+                                     c_int32, c_int32, c_int32, c_float, c_void_p, c_void_p,
+                                     c_void_p, c_void_p, c_size_t, c_void_p]),
     "qsa_get_device_error": (c_int32, [c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
     "qsa_session_create": (c_int32, [ctypes.POINTER(QsaCacheStruct), c_int32, c_int32, c_int32,
                                      c_int32, c_int32, c_int32, c_int32, c_int32, c_float,

@@ -377,6 +377,47 @@ def qsa_index_topk_norm(cache: QSACache, kcn: torch.Tensor, q_idx: torch.Tensor,
                                            _stream(stream)), "qsa_index_topk_norm")
 
 
+def qsa_sparse_prefill_workspace_bytes(n_tokens: int, max_blocks: int, Hq: int, Hkv: int, D: int,
+                                       topk: int) -> int:
+    return int(_lib.load().qsa_sparse_prefill_workspace_bytes(n_tokens, max_blocks, Hq, Hkv, D,
+                                                              topk))
+
+
+def qsa_sparse_prefill(cache: QSACache, cu_q: torch.Tensor, ctx_lens: torch.Tensor,
+                       max_q_per_req: int, q_idx: torch.Tensor, k_chunk: torch.Tensor,
+                       q: torch.Tensor, max_blocks: int, topk: int, sm_scale: float,
+                       sel: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                       workspace: torch.Tensor, stream=None) -> None:
+    """Sparse prefill of the newest n_r tokens of each request (rows cu_q[r]
+    .. cu_q[r+1]-1): every token selects its own blocks over its prefix and
+    attends them.  q [Nq, Hq, D], q_idx / k_chunk [Nq, d] int8, sel
+    [Nq, topk], o [Nq, Hq, D], lse [Nq, Hq]."""
+    Nq, Hq, D = q.shape
+    q_dt = {torch.float32: _lib.QSA_F32, torch.bfloat16: _lib.QSA_BF16}.get(q.dtype)
+    if q_dt is None:
+        raise TypeError("q must be float32 or bfloat16")
+    _need(cu_q, torch.int32, "cu_q")
+    _need(ctx_lens, torch.int32, "ctx_lens")
+    _need(q_idx, torch.int8, "q_idx")
+    _need(k_chunk, torch.int8, "k_chunk")
+    _need(sel, torch.int32, "sel")
+    _need(o, torch.float32, "o")
+    _need(lse, torch.float32, "lse")
+    B = ctx_lens.shape[0]
+    d = cache.ring.shape[-1]
+    if cu_q.shape[0] != B + 1 or q_idx.shape != (Nq, d) or k_chunk.shape != (Nq, d):
+        raise ValueError("cu_q [B+1], q_idx and k_chunk [Nq, d] expected")
+    if sel.shape != (Nq, topk) or o.shape != (Nq, Hq, D) or lse.shape != (Nq, Hq):
+        raise ValueError("sel [Nq, topk], o [Nq, Hq, D] and lse [Nq, Hq] expected")
+    s = cache.struct()
+    _check(_lib.load().qsa_sparse_prefill(ctypes.byref(s), B, Nq, int(max_q_per_req), _ptr(cu_q),
+                                          _ptr(ctx_lens), _ptr(q_idx), _ptr(k_chunk), _ptr(q),
+                                          q_dt, Hq, int(max_blocks), int(topk), float(sm_scale),
+                                          _ptr(sel), _ptr(o), _ptr(lse), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream(stream)), "qsa_sparse_prefill")
+
+
 class QSASession:
     """Decode steps from host buffers to host buffers (qsa_session_*): the
     library owns the device buffers and overlaps each step's uploads and

@@ -14,6 +14,7 @@
 #include "compress_append.cuh"
 #include "index_topk.cuh"
 #include "index_norm.cuh"
+#include "prefill.cuh"
 #include "sparse_decode.cuh"
 #include "sparse_decode_warp.cuh"
 #include "sparse_decode_group.cuh"
@@ -92,6 +93,7 @@ CacheDev to_dev(const qsa_cache *c) {
   d.ring_rows = c->ring_rows;
   d.block_table = c->block_table;
   d.max_pages_per_req = c->max_pages_per_req;
+  d.table_row = nullptr;
   return d;
 }
 
@@ -452,7 +454,8 @@ qsa_status sparse_decode_call(const qsa_cache *cache, int32_t B, int32_t T, int3
                               const int32_t *sel, int32_t topk, float sm_scale, int32_t num_splits,
                               int32_t split_lo, int32_t split_hi, float *o_part, float *lse_part,
                               float *o_merged, float *lse_merged, void *workspace,
-                              size_t workspace_bytes, qsa_stream_t stream) {
+                              size_t workspace_bytes, qsa_stream_t stream,
+                              const int32_t *table_row = nullptr) {
   qsa_status st = check_cache(cache);
   if (st != QSA_OK) return st;
   const int Hkv = cache->num_kv_heads;
@@ -497,6 +500,7 @@ qsa_status sparse_decode_call(const qsa_cache *cache, int32_t B, int32_t T, int3
   const int M = G * T;
   qsa::dec::Params p;
   p.c = to_dev(cache);
+  p.c.table_row = table_row;
   p.B = B;
   p.T = T;
   p.Hq = Hq;
@@ -726,6 +730,143 @@ qsa_status qsa_index_topk_norm(const qsa_cache *cache, const void *kcn, int32_t 
     case 64: return launch_index_topk_norm<64>(sp, s);
     default: return launch_index_topk_norm<128>(sp, s);
   }
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Sparse prefill: many query tokens per request, each with its own selection.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct PrefillLayout {
+  size_t scores, tok_len, tok_row, dec, total;
+};
+
+PrefillLayout prefill_layout(int32_t n_tokens, int32_t max_blocks, int32_t Hq, int32_t Hkv,
+                             int32_t D, int32_t topk) {
+  PrefillLayout l;
+  l.scores = 0;
+  l.tok_len = align_up((size_t)n_tokens * (size_t)max_blocks * sizeof(int32_t));
+  l.tok_row = l.tok_len + align_up((size_t)n_tokens * sizeof(int32_t));
+  l.dec = l.tok_row + align_up((size_t)n_tokens * sizeof(int32_t));
+  l.total = l.dec + qsa_sparse_decode_workspace_bytes(n_tokens, 1, Hq, Hkv, D, topk, 1);
+  return l;
+}
+
+template <int DI>
+qsa_status launch_prefill_scan(const qsa::pre::ScanParams &sp, int B, int max_q, cudaStream_t s) {
+  static bool done[kMaxDevices] = {false};
+  auto kernel = qsa::pre::prefill_scan_kernel<DI>;
+  const size_t smem = qsa::pre::smem_bytes<DI>();
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (prepare_kernel(kernel, smem, done) != cudaSuccess) return QSA_ERR_CUDA;
+  }
+  const dim3 grid((unsigned)((sp.max_blocks + qsa::pre::kBlkPerCta - 1) / qsa::pre::kBlkPerCta),
+                  (unsigned)((max_q + qsa::pre::kTokTile - 1) / qsa::pre::kTokTile), (unsigned)B);
+  return launch(true, kernel, grid, dim3(qsa::pre::kThreads), smem, s, sp);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t qsa_sparse_prefill_workspace_bytes(int32_t n_tokens, int32_t max_blocks, int32_t Hq,
+                                          int32_t Hkv, int32_t D, int32_t topk) {
+  if (n_tokens < 0 || max_blocks < 1 || Hq < 1 || Hkv < 1 || D < 1 || topk < 1) return 0;
+  return prefill_layout(n_tokens, max_blocks, Hq, Hkv, D, topk).total;
+}
+
+qsa_status qsa_sparse_prefill(const qsa_cache *cache, int32_t B, int32_t n_tokens,
+                              int32_t max_q_per_req, const int32_t *cu_q, const int32_t *ctx_lens,
+                              const int8_t *q_idx, const int8_t *k_chunk, const void *q,
+                              int32_t q_dtype, int32_t Hq, int32_t max_blocks, int32_t topk,
+                              float sm_scale, int32_t *sel, float *o, float *lse, void *workspace,
+                              size_t workspace_bytes, qsa_stream_t stream) {
+  qsa_status st = check_cache(cache);
+  if (st != QSA_OK) return st;
+  if (B < 0 || n_tokens < 0 || max_q_per_req < 0) return QSA_ERR_INVALID_ARG;
+  if (topk < 1 || topk > qsa::topk::kMaxTopk) return QSA_ERR_INVALID_ARG;
+  if (max_blocks < 1 || max_blocks > (1 << 24)) return QSA_ERR_INVALID_ARG;
+  if (cache->idx_dim != 32 && cache->idx_dim != 64 && cache->idx_dim != 128)
+    return QSA_ERR_UNSUPPORTED;
+  if (B == 0 || n_tokens == 0) return QSA_OK;
+  if (max_q_per_req < 1 || B > 65535 || n_tokens > 65535 ||
+      (max_q_per_req + qsa::pre::kTokTile - 1) / qsa::pre::kTokTile > 65535)
+    return QSA_ERR_UNSUPPORTED;
+  if (!cu_q || !ctx_lens || !q_idx || !k_chunk || !q || !sel || !o || !lse || !workspace ||
+      !cache->kc)
+    return QSA_ERR_INVALID_ARG;
+  if (!aligned(q_idx, 16) || !aligned(k_chunk, 4) || !aligned(cache->kc, 16) ||
+      !aligned(workspace, 256))
+    return QSA_ERR_INVALID_ARG;
+  const int Hkv = cache->num_kv_heads, D = cache->head_dim;
+  if (Hq < 1 || Hq % Hkv != 0) return QSA_ERR_INVALID_ARG;
+  const PrefillLayout lay = prefill_layout(n_tokens, max_blocks, Hq, Hkv, D, topk);
+  if (workspace_bytes < lay.total) return QSA_ERR_INVALID_ARG;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int32_t *scores = reinterpret_cast<int32_t *>(ws + lay.scores);
+  int32_t *tok_len = reinterpret_cast<int32_t *>(ws + lay.tok_len);
+  int32_t *tok_row = reinterpret_cast<int32_t *>(ws + lay.tok_row);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  // 1. scores of every query token against its prefix blocks (tensor cores)
+  qsa::pre::ScanParams sp;
+  sp.c = to_dev(cache);
+  sp.cu_q = cu_q;
+  sp.ctx_lens = ctx_lens;
+  sp.q_idx = q_idx;
+  sp.max_blocks = max_blocks;
+  sp.n_tok = n_tokens;
+  sp.scores = scores;
+  switch (cache->idx_dim) {
+    case 32: st = launch_prefill_scan<32>(sp, B, max_q_per_req, s); break;
+    case 64: st = launch_prefill_scan<64>(sp, B, max_q_per_req, s); break;
+    default: st = launch_prefill_scan<128>(sp, B, max_q_per_req, s); break;
+  }
+  if (st != QSA_OK) return st;
+  // 2. per-token lengths and rows, own-block fix-up
+  qsa::pre::PrepParams pp;
+  pp.B = B;
+  pp.n_tok = n_tokens;
+  pp.cu_q = cu_q;
+  pp.ctx_lens = ctx_lens;
+  pp.q_idx = q_idx;
+  pp.k_chunk = k_chunk;
+  pp.d = cache->idx_dim;
+  pp.max_blocks = max_blocks;
+  pp.scores = scores;
+  pp.tok_len = tok_len;
+  pp.tok_row = tok_row;
+  st = launch(true, qsa::pre::prefill_prep_kernel, dim3((unsigned)((n_tokens * 32LL + 255) / 256)),
+              dim3(256), 0, s, pp);
+  if (st != QSA_OK) return st;
+  // 3. per-token selection over blocks 0 .. floor(p/4)
+  {
+    static bool done_sel[kMaxDevices] = {false};
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (prepare_kernel(qsa::topk::select_kernel<qsa::topk::IntKeys>, select_smem(), done_sel) !=
+        cudaSuccess)
+      return QSA_ERR_CUDA;
+  }
+  qsa::topk::Params tp;
+  tp.c = to_dev(cache);
+  tp.B = n_tokens;
+  tp.q_idx = q_idx;
+  tp.ctx_lens = tok_len;
+  tp.n_sel = nullptr;
+  tp.max_blocks = max_blocks;
+  tp.topk = topk;
+  tp.sel = sel;
+  tp.scores = scores;
+  st = launch(true, qsa::topk::select_kernel<qsa::topk::IntKeys>, dim3((unsigned)n_tokens),
+              dim3(qsa::topk::kSelThreads), select_smem(), s, tp);
+  if (st != QSA_OK) return st;
+  // 4. attention of every token over its kept tokens (one split: o, lse)
+  return sparse_decode_call(cache, n_tokens, 1, Hq, q, q_dtype, tok_len, sel, topk, sm_scale, 1, 0,
+                            1, o, lse, nullptr, nullptr, ws + lay.dec, lay.total - lay.dec, stream,
+                            tok_row);
 }
 
 }  // extern "C"

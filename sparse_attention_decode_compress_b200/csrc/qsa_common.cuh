@@ -105,6 +105,9 @@ struct CacheDev {
   int ring_rows;
   const int32_t *block_table;
   int max_pages_per_req;
+  // row of block_table of each request, or NULL for row r: the queries of
+  // a prefill share their request's row
+  const int32_t *table_row;
 };
 
 // Physical page of logical page `lp` of request r, or -1 (and an error bit)
@@ -115,7 +118,8 @@ __device__ __forceinline__ int physical_page(const CacheDev &c, int r, long long
     record_error(kErrBounds);
     return -1;
   }
-  const int p = c.block_table[(long long)r * c.max_pages_per_req + lp];
+  const long long row = c.table_row ? (long long)c.table_row[r] : (long long)r;
+  const int p = c.block_table[row * c.max_pages_per_req + lp];
   if (p < 0 || p >= c.num_pages) {
     record_error(kErrBounds);
     return -1;

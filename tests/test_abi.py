@@ -141,3 +141,27 @@ def test_norm_indexer_rejects_bad_arguments_on_the_host():
                                    None, 0x100, 1 << 20, None) == 1
     assert lib.qsa_index_topk_norm(ctypes.byref(c), 0x100, 0, None, None, None, 16, 8, None, None,
                                    None, 0, None) == 0
+
+
+def test_sparse_prefill_rejects_bad_arguments_on_the_host():
+    lib = _lib.load()
+    c = _cache()
+    assert lib.qsa_sparse_prefill_workspace_bytes(0, 16, 16, 2, 128, 8) > 0
+    assert lib.qsa_sparse_prefill_workspace_bytes(4, 0, 16, 2, 128, 8) == 0
+    ok = dict(B=1, n=4, maxq=4, cu=0x100, lens=0x100, qi=0x100, kc=0x100, q=0x100, qd=1, Hq=16,
+              mb=16, topk=8, sm=0.1, sel=0x100, o=0x100, lse=0x100, ws=0x100, wsb=1 << 30)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.qsa_sparse_prefill(ctypes.byref(c), a["B"], a["n"], a["maxq"], a["cu"],
+                                      a["lens"], a["qi"], a["kc"], a["q"], a["qd"], a["Hq"],
+                                      a["mb"], a["topk"], a["sm"], a["sel"], a["o"], a["lse"],
+                                      a["ws"], a["wsb"], None)
+    assert call(topk=0) == 1
+    assert call(mb=0) == 1
+    assert call(qi=0x108) == 1            # indexer queries 16-byte aligned
+    assert call(ws=0x180) == 1            # workspace 256-byte aligned
+    assert call(wsb=16) == 1              # workspace too small
+    assert call(Hq=15) == 1               # Hq % Hkv
+    assert call(n=70000) == 2             # more query tokens than one call takes
+    assert call(B=0) == 0 and call(n=0) == 0   # nothing to do

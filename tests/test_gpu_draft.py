@@ -67,8 +67,8 @@ def _oracle_rows(b, r, L0, S, budget):
                                                 ("mixed_fp8", [4099, 12345], 4, 2048),
                                                 ("mtp_verify", [30001, 5003], 3, 512)])
 def test_draft_steps_reuse_the_step0_selection(name, lens, S, budget):
-    w = replace(WORKLOADS[name], T=4)
-    b = make_batch(w, "cuda", ctx_lens=lens, seed=51)   # final lengths L0 + 3
+    b = make_batch(replace(WORKLOADS[name], T=4), "cuda", ctx_lens=lens, seed=51)  # lengths L0 + 3
+    w = b.w
     B = w.batch
     cache = H.build_cache(b)
     H.prefill(cache, b, 4)                                # positions [0, L0 - 1)

@@ -272,3 +272,27 @@ def norm_indexer_inputs(batch: QSABatch, seed: int = 0, weight_std: float = 0.0)
         weight = torch.randn(w.d_idx, generator=gen, device=device,
                              dtype=torch.float32) * weight_std
     return dict(k=k, q=q, weight=weight)
+
+
+def prefill_inputs(batch: QSABatch, n_q: list[int], seed: int = 0) -> dict:
+    """Inputs of a sparse prefill over `batch`: the newest n_q[r] tokens of
+    request r are its query tokens.  Returns cu_q (int32 [B+1]), their rows
+    in batch.k_idx (the chunk's raw indexer keys), per-token indexer queries
+    q_idx (int8 [Nq, d], uniform in [-127, 127]) and attention queries q
+    ([Nq, Hq, D] of the workload's query dtype, ~ N(0, 1))."""
+    w = batch.w
+    device = batch.device
+    L = batch.ctx_lens_host
+    if len(n_q) != w.batch or any(int(n) > int(l) or n < 0 for n, l in zip(n_q, L.tolist())):
+        raise ValueError("one chunk length per request, at most its context")
+    cu = torch.zeros(w.batch + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(torch.tensor(n_q, dtype=torch.int64), 0)
+    rows = torch.cat([torch.arange(int(batch.cu_ctx_host[r + 1]) - n_q[r],
+                                   int(batch.cu_ctx_host[r + 1])) for r in range(w.batch)])
+    gen = torch.Generator(device=device).manual_seed(seed + 11)
+    nq = int(cu[-1])
+    q_idx = torch.randint(-127, 128, (nq, w.d_idx), generator=gen, device=device, dtype=torch.int8)
+    q = torch.randn((nq, w.Hq, w.D), generator=gen, device=device,
+                    dtype=torch.float32).to(TORCH_DTYPES[w.q_dtype])
+    return dict(cu_q=cu.to(torch.int32), rows=rows, q_idx=q_idx, q=q,
+                k_chunk=batch.k_idx[rows.to(device)].contiguous())
