@@ -53,6 +53,12 @@ def parse_args(argv=None):
                     help="time the steps as eager launches instead of one CUDA graph replay")
     ap.add_argument("--cpu-queries", type=int, default=300,
                     help="oracle queries timed for the CPU baseline")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time the sparse prefill (qsa_sparse_prefill) instead of the decode step")
+    ap.add_argument("--prefill-batch", type=int, default=4)
+    ap.add_argument("--prefill-ctx", type=int, default=32768)
+    ap.add_argument("--prefill-chunk", type=int, default=1024,
+                    help="query tokens per request: the newest tokens of each context")
     return ap.parse_args(argv)
 
 
@@ -179,8 +185,9 @@ def measured_peaks() -> dict:
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
-    return dict(hbm_gbs=6650.0, source="fallback")
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, source="fallback")
 
 
 # ---------------------------------------------------------------------------
@@ -451,11 +458,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             if ev is not None:
                 ev[2].record(stream)
             return
-        qapi.qsa_sparse_decode(cache, batch.q, batch.ctx_lens, step.sel, step.sm_scale, S,
-                               step.o_part, step.lse_part, step.ws_dec)
+        qapi.qsa_sparse_decode_merged(cache, batch.q, batch.ctx_lens, step.sel, step.sm_scale, S,
+                                      step.o_part, step.lse_part, step.o, step.lse, step.ws_dec)
         if ev is not None:
             ev[2].record(stream)
-        qapi.qsa_lse_merge(step.o_part, step.lse_part, step.o, step.lse)
 
     for _ in range(args.warmup):
         one_step()
@@ -604,8 +610,144 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     return line
 
 
+PREFILL_METRIC = "QSA sparse prefill query tokens/s (chunk of the newest tokens, own selection per token)"
+
+
+def prefill_flops(w, L: int, chunk: int, topk: int) -> dict:
+    """Algorithmic work of a prefill chunk of one request: the indexer
+    contraction (2 d int8 operations per token and competing block) and the
+    attention (QK and PV: 4 D FLOPs per head and attended token)."""
+    scan = att = 0
+    for p in range(L - chunk, L):
+        n = p // 4 + 1
+        scan += 2 * w.d_idx * n
+        att += 4 * w.D * w.Hq * min(4 * min(topk, n), p + 1)
+    return dict(scan_int8_ops=scan, attention_flops=att)
+
+
+def run_prefill(args) -> dict:
+    """One step = qsa_compress_append of each request's chunk of indexer keys
+    (an idempotent re-append at the same positions) + qsa_sparse_prefill of
+    the chunk's tokens."""
+    import torch
+    from dataclasses import replace
+    from sparse_attention_decode_compress_b200 import api as qapi
+    from workloads.qsa_inputs import WORKLOADS, make_batch, prefill_inputs
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = replace(WORKLOADS["b32_32k"], name="prefill", batch=args.prefill_batch,
+                ctx=f"fixed:{args.prefill_ctx}", planted=8,
+                description=f"{args.prefill_batch} requests x {args.prefill_ctx} ctx, the newest "
+                            f"{args.prefill_chunk} tokens of each as query tokens, GQA 16/2, D 128, "
+                            f"bf16, page 64 random table, top-512 blocks per token")
+    batch = make_batch(w, dev, seed=5)
+    B, chunk = w.batch, args.prefill_chunk
+    pi = prefill_inputs(batch, [chunk] * B, seed=5)
+    L_host = batch.ctx_lens_host
+    max_blocks = int((L_host.max() + 3) // 4)
+    cache = qapi.QSACache.allocate(batch.k_cache, batch.v_cache, batch.block_table, w.d_idx,
+                                   ring_rows=B)
+    n_pre = L_host - chunk
+    k_pre = torch.cat([batch.k_idx[int(batch.cu_ctx_host[r]): int(batch.cu_ctx_host[r]) + int(n_pre[r])]
+                       for r in range(B)])
+    cu_pre = torch.zeros(B + 1, dtype=torch.int32)
+    cu_pre[1:] = torch.cumsum(n_pre, 0).to(torch.int32)
+    qapi.qsa_compress_append(cache, torch.zeros(B, dtype=torch.int32, device=dev), cu_pre.to(dev),
+                             k_pre, int(n_pre.max()))
+    del k_pre
+    Nq = B * chunk
+    cu_q = pi["cu_q"].to(dev)
+    pos0 = (L_host - chunk).to(torch.int32).to(dev)
+    Hkv, D = batch.k_cache.shape[2], batch.k_cache.shape[3]
+    sel = torch.empty((Nq, w.topk), dtype=torch.int32, device=dev)
+    o = torch.empty((Nq, w.Hq, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((Nq, w.Hq), dtype=torch.float32, device=dev)
+    ws = qapi.new_workspace(qapi.qsa_sparse_prefill_workspace_bytes(Nq, max_blocks, w.Hq, Hkv, D,
+                                                                    w.topk), dev)
+    sm = 1.0 / math.sqrt(D)
+    stream = torch.cuda.current_stream()
+
+    def one_step(ev=None):
+        qapi.qsa_compress_append(cache, pos0, cu_q, pi["k_chunk"], chunk)
+        if ev is not None:
+            ev[0].record(stream)
+        qapi.qsa_sparse_prefill(cache, cu_q, batch.ctx_lens, chunk, pi["q_idx"], pi["k_chunk"],
+                                pi["q"], max_blocks, w.topk, sm, sel, o, lse, ws)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    st, flags = qapi.qsa_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error during warm-up: status {st} flags {flags}")
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)
+    K = args.steps
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cap):
+        for _ in range(K):
+            one_step()
+    graph.replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark("t0")
+    t0.record(stream)
+    graph.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark("t1")
+    ms = t0.elapsed_time(t1)
+    del graph
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    for k in range(K):
+        one_step(evs[k])
+    torch.cuda.synchronize()
+    sampler.mark("t2")
+    pre_ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    st, flags = qapi.qsa_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the timed region: status {st} flags {flags}")
+    clocks = sampler.stop()
+    peaks = measured_peaks()
+    f = [prefill_flops(w, int(L), chunk, w.topk) for L in L_host.tolist()]
+    att = sum(x["attention_flops"] for x in f)
+    scan = sum(x["scan_int8_ops"] for x in f)
+    # bf16-equivalent work: int8 tensor-core operations run at twice the
+    # bf16 rate (nominal 4.5 vs 2.25 PFLOP/s dense)
+    work = att + scan / 2
+    achieved = work / (pre_ms / 1e3) / 1e12
+    return {
+        "metric": PREFILL_METRIC, "value": round(Nq * K / (ms / 1e3), 1), "unit": "tokens/s",
+        "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded)",
+        "config": {"workload": "prefill", "description": w.description, "global_batch": B,
+                   "seq_len": args.prefill_ctx, "query_tokens": chunk, "topk_blocks": w.topk,
+                   "page_size": w.page_size, "parallelism": "single GPU",
+                   "timing": "value: K steps (append + prefill) as one CUDA graph replay; "
+                             "roofline: eager pass with events around the prefill call"},
+        "roofline": {"bound": "tensor", "kernel": "qsa_sparse_prefill (all its kernels)",
+                     "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "peak_source": peaks["source"], "traffic": None,
+                     "launch_ms": round(pre_ms, 5),
+                     "flops_per_launch": {"attention": att, "scan_int8_ops": scan}},
+        "gpu_launches": 6 * K,
+        "clocks": clocks,
+    }
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.prefill and args.impl == "ours":
+        print(json.dumps(run_prefill(args)), flush=True)
+        return 0
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

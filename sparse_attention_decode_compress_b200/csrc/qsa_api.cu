@@ -18,6 +18,7 @@
 #include "sparse_decode.cuh"
 #include "sparse_decode_warp.cuh"
 #include "sparse_decode_group.cuh"
+#include "sparse_decode_streamk.cuh"
 #include "lse_merge.cuh"
 
 namespace {
@@ -291,6 +292,88 @@ qsa_status launch_decode_group(qsa::dec::Params p, cudaStream_t stream) {
   return launch(true, kernel, dim3(ctas), dim3(NW * 32), smem, stream, p);
 }
 
+// ------------------------------------------------------- stream-K decode --
+// Entries per pair in the global list of the stream-K decode; warps of a
+// launch (at most 2048, ranges of at least 16 entries; W_hw = the resident
+// warps of the device); partial slots per (pair, split): a split of at most
+// E entries meets at most ceil(E / l) + 1 warp ranges of l >= floor(X / W)
+// entries, largest for the most warps the launch may use (so the workspace
+// size needs no device).
+int sk_entries(int topk, int T) { return topk + (T > 1 ? 2 : 0); }
+constexpr long long kSKMaxWarps = 2048;
+constexpr long long kSKMinEntries = 16;
+long long sk_warps(long long X, long long w_hw) {
+  return std::max<long long>(1, std::min({w_hw, kSKMaxWarps, X / kSKMinEntries}));
+}
+int sk_slots(long long pairs, int E) {
+  const long long X = pairs * E;
+  const long long l = X / sk_warps(X, kSKMaxWarps);
+  if (l < 1) return 1;  // no entries (B = 0)
+  return (int)((E + l - 1) / l) + 1;
+}
+struct SKLayout {
+  size_t ebound, lse, o, total;
+};
+SKLayout sk_layout(int B, int T, int Hq, int Hkv, int topk, int S, int D) {
+  const long long pairs = (long long)B * Hkv;
+  const int K = sk_slots(pairs, sk_entries(topk, T));
+  const size_t M = (size_t)(Hq / Hkv) * T;
+  SKLayout l;
+  l.ebound = 0;
+  l.lse = align_up((size_t)B * (S + 1) * sizeof(int32_t));
+  l.o = l.lse + align_up((size_t)pairs * S * K * M * sizeof(float));
+  l.total = l.o + align_up((size_t)pairs * S * K * M * D * sizeof(float));
+  return l;
+}
+
+template <int D>
+qsa_status launch_decode_streamk(const qsa::dec::Params &p, float *o, float *lse, void *workspace,
+                                 cudaStream_t stream) {
+  constexpr int NW = kDecWarps;
+  constexpr int NS = kDecStages;
+  static bool done[kMaxDevices] = {false};
+  static int blocks_per_sm[kMaxDevices] = {0};
+  auto kernel = qsa::dec::sparse_decode_streamk_kernel<D, NW, NS>;
+  const size_t smem = sizeof(qsa::dec::WarpSmem<D, false, NW, NS>) + 128;
+  const int dev = current_device();
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (prepare_kernel(kernel, smem, done) != cudaSuccess) return QSA_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices && !blocks_per_sm[dev]) {
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, NW * 32, smem) != cudaSuccess)
+        return QSA_ERR_CUDA;
+      blocks_per_sm[dev] = n > 0 ? n : 1;
+    }
+  }
+  const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
+  qsa::dec::SKParams sk;
+  sk.p = p;
+  sk.p.chunk = 1 << 20;  // the plan's chunk count is not used by this kernel
+  const long long pairs = (long long)p.B * p.c.num_kv_heads;
+  sk.E = sk_entries(p.topk, p.T);
+  sk.X = pairs * sk.E;
+  sk.K = sk_slots(pairs, sk.E);
+  // one wave of resident CTAs at most; warps past W return at once
+  sk.W = (int)sk_warps(sk.X, (long long)bps * sm_count(dev) * NW);
+  const long long ctas = (sk.W + NW - 1) / NW;
+  const SKLayout lay = sk_layout(p.B, p.T, p.Hq, p.c.num_kv_heads, p.topk, p.S, D);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  sk.sk_ebound = reinterpret_cast<int32_t *>(ws + lay.ebound);
+  sk.sk_lse = reinterpret_cast<float *>(ws + lay.lse);
+  sk.sk_o = reinterpret_cast<float *>(ws + lay.o);
+  sk.o = o;
+  sk.lse = lse;
+  qsa_status st = launch(true, kernel, dim3((unsigned)ctas), dim3(NW * 32), smem, stream, sk);
+  if (st != QSA_OK) return st;
+  const long long rows = pairs * p.M;
+  const long long grid = (rows * 32 + qsa::dec::kSKMergeThreads - 1) / qsa::dec::kSKMergeThreads;
+  if (grid > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  auto merge = (p.s_hi - p.s_lo <= 4) ? qsa::dec::streamk_merge_kernel<D, 4>
+                                      : qsa::dec::streamk_merge_kernel<D, qsa::dec::kMaxSplits>;
+  return launch(true, merge, dim3((unsigned)grid), dim3(qsa::dec::kSKMergeThreads), 0, stream, sk);
+}
+
 template <int D, bool FP8>
 qsa_status dispatch_decode_nt(const qsa::dec::Params &p, int NT, cudaStream_t stream) {
   switch (NT) {
@@ -440,7 +523,11 @@ size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32
   // room for the smallest chunks the launch may pick
   const size_t nch = decode_chunk_slots(topk, num_splits, qsa::dec::kMinChunkBlocks);
   const size_t slots = (size_t)B * Hkv * nch;
-  return kTicketBytes + align_up(slots * M * D * sizeof(float)) + align_up(slots * M * sizeof(float));
+  const size_t chunked =
+      kTicketBytes + align_up(slots * M * D * sizeof(float)) + align_up(slots * M * sizeof(float));
+  // the stream-K decode (at most 8 query rows per kv head, bf16 / fp8)
+  const size_t streamk = sk_layout(B, T, Hq, Hkv, topk, num_splits, D).total;
+  return std::max(chunked, streamk);
 }
 
 }  // extern "C"
@@ -479,8 +566,11 @@ qsa_status sparse_decode_call(const qsa_cache *cache, int32_t B, int32_t T, int3
   if (B > 65535 || Hkv > 65535) return QSA_ERR_UNSUPPORTED;
   // cache rows are indexed with 32-bit integers
   if ((long long)cache->num_pages * cache->page_size * Hkv > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
-  if ((size_t)B * Hkv * num_splits * sizeof(int32_t) >
-      kTicketBytes - qsa::dec::kCounterInts * sizeof(int32_t))
+  // bf16 caches with at most 8 query rows per kv head take the stream-K
+  // decode; the rest the chunked decode with its ticket header
+  const bool streamk = cache->kv_dtype == QSA_BF16 && G * T <= 8;
+  if (!streamk && (size_t)B * Hkv * num_splits * sizeof(int32_t) >
+                      kTicketBytes - qsa::dec::kCounterInts * sizeof(int32_t))
     return QSA_ERR_UNSUPPORTED;
   const bool merged = o_merged != nullptr;
   if (merged && (!lse_merged || !aligned(o_merged, 16) || split_lo != 0 || split_hi != num_splits))
@@ -526,6 +616,11 @@ qsa_status sparse_decode_call(const qsa_cache *cache, int32_t B, int32_t T, int3
   p.nch = nch;  // the launch sets nch and chunk for its kernel
   p.chunk = qsa::dec::kMinChunkBlocks;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (streamk) {
+    // decode + merge of its partials (into o_part, and o / lse when merged)
+    return D == 64 ? launch_decode_streamk<64>(p, o_merged, lse_merged, workspace, s)
+                   : launch_decode_streamk<128>(p, o_merged, lse_merged, workspace, s);
+  }
   // the header (work counters, split tickets) starts at zero in every call,
   // whatever the workspace held
   const int header_ints = qsa::dec::kCounterInts + B * Hkv * num_splits;

@@ -40,8 +40,15 @@ class QSADecodeStep:
                                  self.o_part, self.lse_part, self.o, self.lse, self.ws_dec, stream)
         return self.o, self.lse
 
-    # kernels one call launches: append, scan, select, decode, merge
-    kernels_per_step = 5
+    @property
+    def kernels_per_step(self) -> int:
+        """Kernels one step launches: append, scan, select, then the decode
+        and its merge; the chunked decode (float32 or fp8 caches, or more
+        than 8 query rows per kv head) adds the kernel that zeroes its
+        workspace header."""
+        G = self.Hq // self.cache.k_cache.shape[2]
+        chunked = self.cache.k_cache.dtype != torch.bfloat16 or G * self.T > 8
+        return 6 if chunked else 5
 
 
 class QSADraftDecode:
