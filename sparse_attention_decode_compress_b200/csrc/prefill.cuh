@@ -293,9 +293,18 @@ __global__ void __launch_bounds__(kThreads) prefill_scan_kernel(ScanParams sp) {
       tmem_ld_wait();
       if (row < ntok) {
         int32_t *dst = out_rows + (long long)row * sp.max_blocks + bcol0 + c0;
+        int32_t v[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (c0 + e < ncol) dst[e] = (int32_t)a1[e] + 256 * (int32_t)a2[e];
+        for (int e = 0; e < 16; ++e) v[e] = (int32_t)a1[e] + 256 * (int32_t)a2[e];
+        if (c0 + 16 <= ncol && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<int4 *>(dst + e) = make_int4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (c0 + e < ncol) dst[e] = v[e];
+        }
       }
     }
     tc_fence_before();
