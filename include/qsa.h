@@ -168,10 +168,16 @@ size_t qsa_index_topk_workspace_bytes(int32_t B, int32_t max_blocks);
  *   sel      [B, topk] int32 output
  *   scores   [B, max_blocks] int32 output of every score, or NULL
  *   workspace  >= qsa_index_topk_workspace_bytes(B, max_blocks) bytes,
- *            16-byte aligned, any contents (it holds the scores when
- *            `scores` is NULL); calls that overlap on the GPU need separate
- *            workspaces.  Two kernels run: a scan that writes every score,
- *            then a selection with one CTA per request.
+ *            16-byte aligned, any contents: it holds the maxima of the
+ *            scan's groups of 2048/d consecutive blocks, and the scores when
+ *            `scores` is NULL (with `scores` given, 64 KiB + the maxima,
+ *            4 * B * ceil(max_blocks / 16) bytes rounded up to 256, are
+ *            enough); calls that overlap on the GPU need separate
+ *            workspaces.  Two kernels run: a scan that writes every score
+ *            and the group maxima, then a selection with one CTA per
+ *            request, which reads only the groups whose maximum can reach
+ *            the top k (all scores when the request has fewer groups than
+ *            topk).
  * The compressed-key pages are read through the block table.  Errors:
  * QSA_ERR_INVALID_ARG (null pointer, topk or max_blocks out of range,
  * workspace too small or misaligned, kc not 16-byte aligned).

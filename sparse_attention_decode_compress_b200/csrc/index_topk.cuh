@@ -53,7 +53,17 @@ struct Params {
   int32_t *tokens = nullptr;  // [B, 4 * topk] kept token indices (token-budget output), or NULL
   int T = 1;                  // query tokens per request: tokens are listed up to p0 = L - T
   int32_t *scores;   // [B, max_blocks]
+  // maxima of the scan's groups of gsize consecutive rows ([B, max_groups],
+  // max_groups = ceil(max_blocks / gsize)), or NULL: the selection then
+  // reads every score twice
+  int32_t *gmax = nullptr;
+  int gsize = 0;
 };
+
+// Rows per group maximum of the integer scan (one run of a lane's loads
+// across the rows of a load instruction): 16, 32, 64 rows for d = 128, 64, 32.
+template <int DI>
+__host__ __device__ constexpr int scan_group_rows() { return 2048 / DI; }
 
 // Competing blocks of request r, validated the same way in every thread:
 // n = n_sel[r] (or ceil(L/4)), clipped to [0, min(ceil(L/4), max_blocks)].
@@ -109,12 +119,17 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelBatch = 8;  // int4 loads in flight per thread
 constexpr int kBitmapWords = 8192;  // requests of <= 262,144 blocks mark kept blocks in a bitmap
 
+constexpr int kQGroups = 2048;  // groups whose maximum reaches the bound, held in shared memory
+constexpr int kQCand = 2048;    // their scores that reach it
+
 struct SelSmem {
   int hist[kHistBins];  // also the kept-index list (kMaxTopk ints) on the list path
   unsigned long long cand[kCandCap];
   uint32_t bits[kBitmapWords];  // bit i: block i kept
+  int qg[kQGroups];
+  unsigned long long qc[kQCand];  // (~key << 32 | block) of the scores that reach the bound
   int warp_tot[kSelThreads / 32];
-  int bin, above, nkeep, ncand, fb_key, fb_above, fb_idx;
+  int bin, above, nkeep, ncand, fb_key, fb_above, fb_idx, nq, nqc;
 };
 
 // Sum of the per-warp totals sm.warp_tot[0 .. w) (all 32 written before a
@@ -482,6 +497,127 @@ __device__ void select_passes(const int32_t *sc, int n, int K, bool use_bits, Se
   __syncthreads();
 }
 
+// Selection from the group maxima (integer keys, requests of the bitmap
+// path): sets the K kept blocks in sm.bits and returns true, or returns
+// false (the caller then runs the two full passes) when the request has
+// fewer groups than K or the qualifying groups, their qualifying scores or
+// the threshold bin's candidates overflow shared memory.
+//
+// Exact: let L be the lower edge of the histogram bin holding the K-th
+// largest group maximum.  At least K groups have a maximum >= L, so at
+// least K distinct blocks score >= L, so the K-th largest score t_K >= L.
+// Every block of the top K (score >= t_K) therefore lies in a group whose
+// maximum is >= L and scores >= L itself: those blocks are the only
+// candidates, and the histogram / keep passes then run on them in shared
+// memory.  Reads ~16 KB of maxima and the qualifying groups' rows (~1/8 of
+// the row at 65,536 blocks) instead of the whole row twice.
+__device__ bool select_by_group_maxima(const int32_t *sc, const int32_t *gm, int gsize, int n, int K,
+                                       SelSmem &sm, int tid) {
+  constexpr int kShift1 = IntKeys::kBits - 13;
+  const int lane = tid & 31;
+  const int ng = (n + gsize - 1) / gsize;
+  if (ng < K) return false;
+  // A: histogram of the group maxima, the bin of the K-th largest
+  for (int g0 = 0; g0 < ng; g0 += kSelThreads * 4) {
+    int v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int g = g0 + j * kSelThreads + tid;
+      v[j] = g < ng ? __ldcg(gm + g) : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (g0 + j * kSelThreads + tid < ng) atomicAdd(&sm.hist[IntKeys::key(v[j]) >> kShift1], 1);
+  }
+  __syncthreads();
+  find_rank_bin_desc(sm.hist, K, sm, tid);
+  const uint32_t bmax = (uint32_t)sm.bin;
+  // B: the groups whose maximum reaches that bin
+  for (int g0 = 0; g0 < ng; g0 += kSelThreads) {
+    const int g = g0 + tid;
+    const bool q = g < ng && (IntKeys::key(__ldcg(gm + g)) >> kShift1) >= bmax;
+    const unsigned bal = __ballot_sync(0xffffffffu, q);
+    int base = 0;
+    if (lane == 0 && bal) base = atomicAdd(&sm.nq, __popc(bal));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (q) {
+      const int slot = base + __popc(bal & ((1u << lane) - 1u));
+      if (slot < kQGroups) sm.qg[slot] = g;
+    }
+  }
+  for (int i = tid; i < kHistBins; i += kSelThreads) sm.hist[i] = 0;
+  __syncthreads();
+  const int nq = sm.nq;
+  if (nq > kQGroups) return false;
+  // C: the qualifying groups' scores that reach the bin, as (~key, block)
+  const int nv = nq * gsize / 4;
+  for (int e0 = 0; e0 < nv; e0 += kSelThreads * 4) {
+    int4 v[4];
+    int rowv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + j * kSelThreads + tid;
+      rowv[j] = -1;
+      v[j] = make_int4(INT_MIN, INT_MIN, INT_MIN, INT_MIN);
+      if (e < nv) {
+        const int row = sm.qg[(4 * e) / gsize] * gsize + (4 * e) % gsize;
+        const int32_t *src = sc + row;
+        rowv[j] = row;
+        if (row + 3 < n && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+          v[j] = __ldcg(reinterpret_cast<const int4 *>(src));
+        } else {  // a row stride that is not a multiple of 4, or the request's last rows
+          v[j] = make_int4(row < n ? __ldcg(src) : INT_MIN, row + 1 < n ? __ldcg(src + 1) : INT_MIN,
+                           row + 2 < n ? __ldcg(src + 2) : INT_MIN,
+                           row + 3 < n ? __ldcg(src + 3) : INT_MIN);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int sv = c == 0 ? v[j].x : c == 1 ? v[j].y : c == 2 ? v[j].z : v[j].w;
+        const int row = rowv[j] + c;
+        const uint32_t k = IntKeys::key(sv);
+        const bool take = rowv[j] >= 0 && row < n && (k >> kShift1) >= bmax;
+        const unsigned bal = __ballot_sync(0xffffffffu, take);
+        int base = 0;
+        if (lane == 0 && bal) base = atomicAdd(&sm.nqc, __popc(bal));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (take) {
+          const int slot = base + __popc(bal & ((1u << lane) - 1u));
+          if (slot < kQCand) sm.qc[slot] = ((unsigned long long)(0xffffffffu - k) << 32) | (uint32_t)row;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int nc = sm.nqc;
+  if (nc > kQCand) return false;
+  // D: histogram of the candidates, the threshold bin, keep the blocks above
+  // it, gather the bin's blocks
+  for (int i = tid; i < nc; i += kSelThreads)
+    atomicAdd(&sm.hist[(0xffffffffu - (uint32_t)(sm.qc[i] >> 32)) >> kShift1], 1);
+  __syncthreads();
+  find_rank_bin_desc(sm.hist, K, sm, tid);
+  const uint32_t b1 = (uint32_t)sm.bin;
+  for (int i0 = 0; i0 < nc; i0 += kSelThreads) {
+    const int i = i0 + tid;
+    bool take = false;
+    unsigned long long x = 0;
+    if (i < nc) {
+      x = sm.qc[i];
+      const uint32_t d1 = (0xffffffffu - (uint32_t)(x >> 32)) >> kShift1;
+      const int blk = (int)(uint32_t)(x & 0xffffffffu);
+      if (d1 > b1) atomicOr(&sm.bits[blk >> 5], 1u << (blk & 31));
+      take = d1 == b1;
+    }
+    append_cand(take, x, sm);
+  }
+  __syncthreads();
+  return sm.ncand <= kCandCap;
+}
+
 // Selection kernel: grid = B, one request per CTA.
 template <typename KT>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
@@ -515,25 +651,62 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
   if (tid == 0) {
     sm.nkeep = 0;
     sm.ncand = 0;
+    sm.nq = 0;
+    sm.nqc = 0;
   }
   __syncthreads();
-  select_passes<KT>(sc, n, K, use_bits, sm, tid);
+  bool done = false;
+  if constexpr (KT::kBits == IntKeys::kBits) {
+    if (p.gmax && use_bits) {
+      done = select_by_group_maxima(sc, p.gmax + (long long)r * ((p.max_blocks + p.gsize - 1) / p.gsize),
+                                    p.gsize, n, K, sm, tid);
+      if (!done) {  // start over with the two full passes
+        for (int i = tid; i < kHistBins; i += kSelThreads) sm.hist[i] = 0;
+        for (int i = tid; i < nwords; i += kSelThreads) sm.bits[i] = 0u;
+        if (tid == 0) {
+          sm.nkeep = 0;
+          sm.ncand = 0;
+        }
+        __syncthreads();
+      }
+    }
+  }
+  if (!done) select_passes<KT>(sc, n, K, use_bits, sm, tid);
   int *keep = sm.hist;
   const int above = sm.above;
   const int ncand = sm.ncand;
   if (ncand <= kCandCap) {
     // candidates of the threshold bin: the (K - above) first by (score desc,
     // index asc); keys are distinct, so a candidate's rank is the number of
-    // smaller keys
+    // smaller keys.  Few candidates (the usual ~50): every thread compares
+    // a few (i, j) pairs and the ranks are summed in shared memory (in
+    // sm.qg, idle now); many: one thread per candidate counts its rank.
     const int need = K - above;
-    for (int i = tid; i < ncand; i += kSelThreads) {
-      const unsigned long long x = sm.cand[i];
-      int rank = 0;
-      for (int j = 0; j < ncand; ++j) rank += (sm.cand[j] < x);
-      if (rank < need) {
-        const int idx = (int)(uint32_t)(x & 0xffffffffu);
-        if (use_bits) atomicOr(&sm.bits[idx >> 5], 1u << (idx & 31));
-        else keep[above + rank] = idx;
+    if (use_bits && ncand <= 128) {
+      int *rank = sm.qg;
+      for (int i = tid; i < ncand; i += kSelThreads) rank[i] = 0;
+      __syncthreads();
+      for (int pij = tid; pij < ncand * ncand; pij += kSelThreads) {
+        const int i = pij / ncand, j = pij - i * ncand;
+        if (sm.cand[j] < sm.cand[i]) atomicAdd(&rank[i], 1);
+      }
+      __syncthreads();
+      for (int i = tid; i < ncand; i += kSelThreads) {
+        if (rank[i] < need) {
+          const int idx = (int)(uint32_t)(sm.cand[i] & 0xffffffffu);
+          atomicOr(&sm.bits[idx >> 5], 1u << (idx & 31));
+        }
+      }
+    } else {
+      for (int i = tid; i < ncand; i += kSelThreads) {
+        const unsigned long long x = sm.cand[i];
+        int rank = 0;
+        for (int j = 0; j < ncand; ++j) rank += (sm.cand[j] < x);
+        if (rank < need) {
+          const int idx = (int)(uint32_t)(x & 0xffffffffu);
+          if (use_bits) atomicOr(&sm.bits[idx >> 5], 1u << (idx & 31));
+          else keep[above + rank] = idx;
+        }
       }
     }
     __syncthreads();
@@ -855,6 +1028,39 @@ __global__ void __launch_bounds__(kScanThreads, kScanMinCtas) index_scan_kernel(
       } else {
         if (row < n) score_store(dst, acc[k] + qbias, pol_keep);
         if (row + 1 < n) score_store(dst + 1, acc[k + 1] + qbias, pol_keep);
+      }
+    }
+    if (p.gmax) {
+      // maxima of the item's groups of kRunStride rows (one run of every
+      // lane group): a lane's values lie in at most two runs, and the lanes
+      // sharing a run differ only in the lane bits of the xor masks below
+      constexpr int kGroups = kRowsPerItem / kRunStride;
+      const int i0 = (lane % kLPR) << (4 - kR);
+      const int u0 = i0 / kRun;
+      int gmx[2] = {INT_MIN, INT_MIN};
+#pragma unroll
+      for (int k = 0; k < kVals; ++k) {
+        const int i = i0 | k;
+        const int row = row0 + (i / kRun) * kRunStride + kRun * grp + (i % kRun);
+        if (row < n) gmx[i / kRun - u0] = max(gmx[i / kRun - u0], acc[k] + qbias);
+      }
+      constexpr unsigned kShare = (kLPR == 8) ? (1u | 8u | 16u) : (kLPR == 4) ? (4u | 8u | 16u)
+                                                                              : (2u | 4u | 8u | 16u);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        if (kShare & o) {
+          gmx[0] = max(gmx[0], __shfl_xor_sync(0xffffffffu, gmx[0], o));
+          if (kVals > kRun) gmx[1] = max(gmx[1], __shfl_xor_sync(0xffffffffu, gmx[1], o));
+        }
+      }
+      if ((lane & kShare) == 0) {
+        const int mg = (p.max_blocks + kRunStride - 1) / kRunStride;
+        int32_t *gd = p.gmax + (long long)r * mg + row0 / kRunStride;
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const int u = u0 + v;
+          if (v * kRun < kVals && u < kGroups && row0 + u * kRunStride < n) score_store(gd + u, gmx[v], pol_keep);
+        }
       }
     }
     if (!more) break;

@@ -27,13 +27,19 @@ using qsa::CacheDev;
 
 constexpr size_t kAlign = 256;
 // Both workspaces start with a header of this many bytes (the layout does
-// not depend on the call's sizes).  The decode keeps its work counters and
-// split tickets there and zeroes them at the start of every call; the
-// indexer leaves it unused.
+// not depend on the call's sizes).  The chunked decode keeps its work
+// counters and split tickets there and zeroes them at the start of every
+// call; the indexer leaves it unused (its group maxima and scores follow).
 constexpr size_t kTicketBytes = 64 * 1024;
 constexpr int kMaxDevices = 64;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// The indexer's group maxima (one per 2048 / d rows of a request; sized for
+// the smallest groups, d = 128), after the workspace header.
+size_t index_gmax_bytes(long long B, long long max_blocks) {
+  return align_up((size_t)B * (size_t)((max_blocks + 15) / 16) * sizeof(int32_t));
+}
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -43,11 +49,12 @@ qsa_status launch_status() {
 }
 
 // Launches a library kernel; `programmatic` sets programmatic stream
-// serialisation (every kernel opens with pdl_open(), see qsa_common.cuh).
-// Scan, selection, decode and merge take it.  compress_append, which opens
-// a decode step, does not: launched early it pulled the next step's
-// persistent scan into the tail of the previous step's merge, and steps
-// measured ~12% slower on B200.
+// serialisation (every kernel opens with pdl_open() or pdl_wait(), see
+// qsa_common.cuh).  compress_append, which opens a decode step, opens with
+// the wait alone: it launches early behind the previous kernel, but lets the
+// next step's persistent scan launch only when it ends.  (With pdl_open()
+// it pulled the scan into the tail of the previous step's merge, and steps
+// measured ~12% slower on B200.)
 template <typename... KArgs, typename... Args>
 qsa_status launch(bool programmatic, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                   cudaStream_t s, Args... args) {
@@ -436,16 +443,17 @@ qsa_status qsa_compress_append(const qsa_cache *cache, int32_t B, const int32_t 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const dim3 block(qsa::kAppendThreads);
   switch (cache->idx_dim) {
-    case 32: return launch(false, qsa::compress_append_kernel<32>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
-    case 64: return launch(false, qsa::compress_append_kernel<64>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
-    case 128: return launch(false, qsa::compress_append_kernel<128>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
+    case 32: return launch(true, qsa::compress_append_kernel<32>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
+    case 64: return launch(true, qsa::compress_append_kernel<64>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
+    case 128: return launch(true, qsa::compress_append_kernel<128>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
     default: return QSA_ERR_UNSUPPORTED;
   }
 }
 
 size_t qsa_index_topk_workspace_bytes(int32_t B, int32_t max_blocks) {
   if (B < 0 || max_blocks < 0) return 0;
-  return kTicketBytes + align_up((size_t)B * (size_t)max_blocks * sizeof(int32_t));
+  return kTicketBytes + index_gmax_bytes(B, max_blocks) +
+         align_up((size_t)B * (size_t)max_blocks * sizeof(int32_t));
 }
 
 }  // extern "C"
@@ -473,9 +481,11 @@ qsa_status index_topk_call(const qsa_cache *cache, int32_t B, const int8_t *q_id
   if (!aligned(cache->kc, 16) || !aligned(q_idx, 4) || !aligned(workspace, 16) ||
       (scores && !aligned(scores, 4)) || (tokens && !aligned(tokens, 16)))
     return QSA_ERR_INVALID_ARG;
-  const size_t need = scores ? kTicketBytes : qsa_index_topk_workspace_bytes(B, max_blocks);
+  const size_t gmax_bytes = index_gmax_bytes(B, max_blocks);
+  const size_t need = scores ? kTicketBytes + gmax_bytes : qsa_index_topk_workspace_bytes(B, max_blocks);
   if (workspace_bytes < need) return QSA_ERR_INVALID_ARG;
 
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
   qsa::topk::Params p;
   p.c = to_dev(cache);
   p.B = B;
@@ -487,8 +497,9 @@ qsa_status index_topk_call(const qsa_cache *cache, int32_t B, const int8_t *q_id
   p.sel = sel;
   p.tokens = tokens;
   p.T = T;
-  p.scores = scores ? scores
-                    : reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + kTicketBytes);
+  p.scores = scores ? scores : reinterpret_cast<int32_t *>(ws + kTicketBytes + gmax_bytes);
+  p.gmax = reinterpret_cast<int32_t *>(ws + kTicketBytes);
+  p.gsize = 2048 / cache->idx_dim;
   return dispatch_index_topk(p, cache->idx_dim, cache->page_size,
                              reinterpret_cast<cudaStream_t>(stream));
 }
@@ -782,9 +793,9 @@ qsa_status qsa_compress_append_norm(const qsa_cache *cache, void *kcn, void *rin
   const dim3 grid((unsigned)gx, (unsigned)B), block(qsa::norm::kAppendThreads);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (cache->idx_dim) {
-    case 32: return launch(false, qsa::norm::compress_append_norm_kernel<32>, grid, block, 0, s, a);
-    case 64: return launch(false, qsa::norm::compress_append_norm_kernel<64>, grid, block, 0, s, a);
-    default: return launch(false, qsa::norm::compress_append_norm_kernel<128>, grid, block, 0, s, a);
+    case 32: return launch(true, qsa::norm::compress_append_norm_kernel<32>, grid, block, 0, s, a);
+    case 64: return launch(true, qsa::norm::compress_append_norm_kernel<64>, grid, block, 0, s, a);
+    default: return launch(true, qsa::norm::compress_append_norm_kernel<128>, grid, block, 0, s, a);
   }
 }
 

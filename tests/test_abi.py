@@ -43,7 +43,8 @@ def test_status_strings_and_version():
 def test_workspace_sizes():
     lib = _lib.load()
     tick = 64 * 1024
-    assert lib.qsa_index_topk_workspace_bytes(128, 65536) == tick + 128 * 65536 * 4
+    # header, the group maxima (one per 16 blocks), the scores
+    assert lib.qsa_index_topk_workspace_bytes(128, 65536) == tick + 128 * 4096 * 4 + 128 * 65536 * 4
     assert lib.qsa_index_topk_workspace_bytes(-1, 3) == 0
     # decode: B*Hkv*nch slots of (M*D floats + M floats), nch = ceil((topk+2)/32) + S - 1
     # (room for the smallest chunks, 32 micro-blocks, a launch may pick)
