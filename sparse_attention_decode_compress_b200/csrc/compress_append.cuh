@@ -27,7 +27,7 @@ template <int DI>
 __global__ void __launch_bounds__(kAppendThreads) compress_append_kernel(
     CacheDev c, int B, const int32_t *__restrict__ pos0, const int32_t *__restrict__ cu_new,
     const int8_t *__restrict__ k_new, int max_new) {
-  pdl_wait();
+  pdl_open();
   constexpr int kThreadsPerRow = DI / 16;
   constexpr int kRowsPerIter = kAppendThreads / kThreadsPerRow;
   const int r = blockIdx.y;

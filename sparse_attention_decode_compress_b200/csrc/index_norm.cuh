@@ -57,7 +57,7 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8]) {
 
 template <int DI>
 __global__ void __launch_bounds__(kAppendThreads) compress_append_norm_kernel(AppendParams a) {
-  pdl_wait();
+  pdl_open();
   constexpr int kG = DI / 8;  // threads per block row
   constexpr int kRowsPerIter = kAppendThreads / kG;
   const CacheDev &c = a.c;

@@ -49,12 +49,13 @@ qsa_status launch_status() {
 }
 
 // Launches a library kernel; `programmatic` sets programmatic stream
-// serialisation (every kernel opens with pdl_open() or pdl_wait(), see
-// qsa_common.cuh).  compress_append, which opens a decode step, opens with
-// the wait alone: it launches early behind the previous kernel, but lets the
-// next step's persistent scan launch only when it ends.  (With pdl_open()
-// it pulled the scan into the tail of the previous step's merge, and steps
-// measured ~12% slower on B200.)
+// serialisation (every kernel opens with pdl_open(), see qsa_common.cuh).
+// Scan, selection, decode and merge take it.  compress_append, which opens
+// a decode step, does not: launched early it pulled the next step's
+// persistent scan into the tail of the previous step's merge, and steps
+// measured ~12% slower on B200.  (Launched early with only the wait, so
+// that the scan follows it only when it ends, the 256k step still measured
+// ~2 us slower.)
 template <typename... KArgs, typename... Args>
 qsa_status launch(bool programmatic, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                   cudaStream_t s, Args... args) {
@@ -443,9 +444,9 @@ qsa_status qsa_compress_append(const qsa_cache *cache, int32_t B, const int32_t 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const dim3 block(qsa::kAppendThreads);
   switch (cache->idx_dim) {
-    case 32: return launch(true, qsa::compress_append_kernel<32>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
-    case 64: return launch(true, qsa::compress_append_kernel<64>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
-    case 128: return launch(true, qsa::compress_append_kernel<128>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
+    case 32: return launch(false, qsa::compress_append_kernel<32>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
+    case 64: return launch(false, qsa::compress_append_kernel<64>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
+    case 128: return launch(false, qsa::compress_append_kernel<128>, grid, block, 0, s, c, B, pos0, cu_new, k_new, max_new_per_req);
     default: return QSA_ERR_UNSUPPORTED;
   }
 }
@@ -793,9 +794,9 @@ qsa_status qsa_compress_append_norm(const qsa_cache *cache, void *kcn, void *rin
   const dim3 grid((unsigned)gx, (unsigned)B), block(qsa::norm::kAppendThreads);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (cache->idx_dim) {
-    case 32: return launch(true, qsa::norm::compress_append_norm_kernel<32>, grid, block, 0, s, a);
-    case 64: return launch(true, qsa::norm::compress_append_norm_kernel<64>, grid, block, 0, s, a);
-    default: return launch(true, qsa::norm::compress_append_norm_kernel<128>, grid, block, 0, s, a);
+    case 32: return launch(false, qsa::norm::compress_append_norm_kernel<32>, grid, block, 0, s, a);
+    case 64: return launch(false, qsa::norm::compress_append_norm_kernel<64>, grid, block, 0, s, a);
+    default: return launch(false, qsa::norm::compress_append_norm_kernel<128>, grid, block, 0, s, a);
   }
 }
 

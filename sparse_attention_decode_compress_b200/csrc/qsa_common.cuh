@@ -23,8 +23,9 @@ __device__ uint32_t g_error_flags;
 
 __device__ __forceinline__ void record_error(uint32_t bits) { atomicOr(&g_error_flags, bits); }
 
-// Programmatic dependent launch.  The library launches its kernels with
-// programmatic stream serialisation: such a kernel may be
+// Programmatic dependent launch.  The library launches its kernels (all
+// but compress_append, see qsa_api.cu) with programmatic stream
+// serialisation: such a kernel may be
 // scheduled once every CTA of the kernel before it has started, so its
 // CTAs are resident, past their launch, when that kernel ends.  Every kernel
 // opens with pdl_open() before anything else: it lets the next kernel
@@ -35,11 +36,6 @@ __device__ __forceinline__ void pdl_open() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
-// The wait alone: the next kernel launches only when this one ends (the
-// kernel that opens a decode step uses it, so that it launches early behind
-// the previous kernel without letting the next step's persistent kernels in
-// before it is done).
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
