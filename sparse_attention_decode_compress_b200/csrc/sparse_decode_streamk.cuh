@@ -23,6 +23,11 @@
 // 63 + 5.4 us (+ the header reset) for the chunked kernel.  The fp8 decode
 // keeps the chunked kernel: its warps would meet 3-4 split boundaries each,
 // and the restarts and the larger merge cost more than the balance gains.
+// A warp whose range crosses a split or pair boundary restarts its ring
+// there (~3 us).  Streaming a warp's segments back to back instead (one
+// metadata piece per request, segments padded to whole stages, the partial
+// written between stages) measured slower: 64.9 against 57.5 us per launch
+// at batch 128 x 16k, with 3.5x the instruction-fetch stalls.
 #pragma once
 #include "sparse_decode_warp.cuh"
 
@@ -289,11 +294,16 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_streamk_kernel(SKPar
 // o = 0, lse = -inf).  With `o` set, the row's splits are then merged into
 // o / lse with the operations of merge_row (qsa_lse_merge), on the values
 // just computed, so the result has the same bits as qsa_lse_merge of o_part.
-// Three rounds of loads per row: the split boundaries; every slot's lse
-// (the (split, slot) pairs of the row flattened across the lanes); every
-// slot's output row (a float4 slice per lane, all slots at once).
+// The (split, slot) pairs of the row are flattened across the lanes: a
+// first pass over their lse takes each split's maximum, a second weighs
+// every slot by exp(lse - maximum) (lane-parallel) and sums the weights and
+// the weighted rows (a float4 slice per lane, 16 slot rows loaded
+// together) in slot order, so a split's bits do not depend on the lanes its
+// slots land on (which depend on the splits a call computes).  (A running maximum with a rescale per
+// slot, serial over the slots, cost ~60 instructions per slot: 15 us per
+// launch at batch 16 with ~32 slots per split, 8.6 us at batch 128.)
 constexpr int kSKMergeThreads = 128;
-constexpr int kSKMergeSlots = 16;  // (split, slot) pairs handled per round
+constexpr int kSKMergeSlots = 16;  // slot rows loaded together
 
 template <int D, int NSMAX>
 __global__ void __launch_bounds__(kSKMergeThreads) streamk_merge_kernel(SKParams sk) {
@@ -331,18 +341,10 @@ __global__ void __launch_bounds__(kSKMergeThreads) streamk_merge_kernel(SKParams
   }
   first -= nk;
   const int total = __shfl_sync(0xffffffffu, first + nk, 31);
-  float4 os[NSMAX];
-  float mxs[NSMAX], dens[NSMAX];
-#pragma unroll
-  for (int i = 0; i < NSMAX; ++i) {
-    os[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    mxs[i] = -INFINITY;
-    dens[i] = 0.f;
-  }
-  for (int base = 0; base < total; base += kSKMergeSlots) {
-    // lane j: flattened pair base + j -> (split i, slot k), its lse
-    const int f = base + lane;
-    int si = -1, kk = 0;
+  // flattened index f -> (split i, slot) and that slot's lse
+  auto locate = [&](int f, int &si, long long &slot) {
+    si = -1;
+    int kk = 0;
 #pragma unroll
     for (int i = 0; i < NSMAX; ++i) {
       const int fi = __shfl_sync(0xffffffffu, first, i);
@@ -352,37 +354,70 @@ __global__ void __launch_bounds__(kSKMergeThreads) streamk_merge_kernel(SKParams
         kk = f - fi;
       }
     }
-    const long long slot = (P * p.S + p.s_lo + si) * sk.K + kk;
-    const float lv = (si >= 0 && f < total) ? __ldcg(sk.sk_lse + slot * p.M + m) : -INFINITY;
-    // every slot row of this round, a float4 slice per lane, loaded together
-    float4 v[kSKMergeSlots];
-    const int nround = min(kSKMergeSlots, total - base);
+    slot = (P * p.S + p.s_lo + max(si, 0)) * sk.K + kk;
+  };
+  // pass 1: each split's maximum lse
+  float mxs[NSMAX];
 #pragma unroll
-    for (int j = 0; j < kSKMergeSlots; ++j) {
-      const long long sj = __shfl_sync(0xffffffffu, slot, j);
-      v[j] = (j < nround && d < D)
-                 ? __ldcg(reinterpret_cast<const float4 *>(sk.sk_o + (sj * p.M + m) * D + d))
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < NSMAX; ++i) mxs[i] = -INFINITY;
+  for (int base = 0; base < total; base += 32) {
+    int si;
+    long long slot;
+    locate(base + lane, si, slot);
+    const float lv = (si >= 0) ? __ldcg(sk.sk_lse + slot * p.M + m) : -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NSMAX; ++i) {
+      if (i >= ns) break;
+      float x = (si == i) ? lv : -INFINITY;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+      mxs[i] = fmaxf(mxs[i], x);
     }
-    // per split: running max and rescaled sums over this round's slots
+  }
+  // pass 2: weights, their sums and the weighted rows
+  float4 os[NSMAX];
+  float dens[NSMAX];
 #pragma unroll
-    for (int j = 0; j < kSKMergeSlots; ++j) {
-      if (j >= nround) break;
-      const int i = __shfl_sync(0xffffffffu, si, j);
-      const float l = __shfl_sync(0xffffffffu, lv, j);
-      if (l == -INFINITY) continue;
+  for (int i = 0; i < NSMAX; ++i) {
+    os[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    dens[i] = 0.f;
+  }
+  for (int base = 0; base < total; base += 32) {
+    int si;
+    long long slot;
+    locate(base + lane, si, slot);
+    const float lv = (si >= 0) ? __ldcg(sk.sk_lse + slot * p.M + m) : -INFINITY;
+    float mx = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < NSMAX; ++q) {
-        if (q != i) continue;
-        const float nm = fmaxf(mxs[q], l);
-        const float a = (mxs[q] == -INFINITY) ? 0.f : __expf(mxs[q] - nm);
-        const float b = __expf(l - nm);
-        os[q].x = os[q].x * a + b * v[j].x;
-        os[q].y = os[q].y * a + b * v[j].y;
-        os[q].z = os[q].z * a + b * v[j].z;
-        os[q].w = os[q].w * a + b * v[j].w;
-        dens[q] = dens[q] * a + b;
-        mxs[q] = nm;
+    for (int i = 0; i < NSMAX; ++i)
+      if (i == si) mx = mxs[i];
+    const float wgt = (lv == -INFINITY) ? 0.f : __expf(lv - mx);
+    const int nb = min(32, total - base);
+    for (int sub = 0; sub < nb; sub += kSKMergeSlots) {
+      float4 v[kSKMergeSlots];
+      const int nround = min(kSKMergeSlots, nb - sub);
+#pragma unroll
+      for (int j = 0; j < kSKMergeSlots; ++j) {
+        const long long sj = __shfl_sync(0xffffffffu, slot, sub + j);
+        v[j] = (j < nround && d < D)
+                   ? __ldcg(reinterpret_cast<const float4 *>(sk.sk_o + (sj * p.M + m) * D + d))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < kSKMergeSlots; ++j) {
+        if (j >= nround) break;
+        const int i = __shfl_sync(0xffffffffu, si, sub + j);
+        const float w = __shfl_sync(0xffffffffu, wgt, sub + j);
+        if (w == 0.f) continue;  // an empty segment (or an unwritten slot) adds nothing
+#pragma unroll
+        for (int q = 0; q < NSMAX; ++q) {
+          if (q != i) continue;
+          dens[q] += w;
+          os[q].x = __fmaf_rn(w, v[j].x, os[q].x);
+          os[q].y = __fmaf_rn(w, v[j].y, os[q].y);
+          os[q].z = __fmaf_rn(w, v[j].z, os[q].z);
+          os[q].w = __fmaf_rn(w, v[j].w, os[q].w);
+        }
       }
     }
   }
