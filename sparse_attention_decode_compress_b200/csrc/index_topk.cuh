@@ -520,39 +520,63 @@ __device__ bool select_by_group_maxima(const int32_t *sc, const int32_t *gm, int
   const int lane = tid & 31;
   const int ng = (n + gsize - 1) / gsize;
   if (ng < 2 * K) return false;
-  // A: histogram of the group maxima, the bin of the K-th largest
+  // A: histogram of the group maxima, the bin of the K-th largest.  Group
+  // g0 + j * kSelThreads + tid is this thread's j-th; with at most
+  // 4 * kSelThreads groups their maxima stay in registers for B.
+  const bool held = ng <= 4 * kSelThreads;
+  int vh[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
   for (int g0 = 0; g0 < ng; g0 += kSelThreads * 4) {
     int v[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int g = g0 + j * kSelThreads + tid;
-      v[j] = g < ng ? __ldcg(gm + g) : 0;
+      v[j] = g < ng ? __ldcg(gm + g) : INT_MIN;
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < 4; ++j) {
       if (g0 + j * kSelThreads + tid < ng) atomicAdd(&sm.hist[IntKeys::key(v[j]) >> kShift1], 1);
+      vh[j] = v[j];
+    }
   }
   __syncthreads();
   find_rank_bin_desc(sm.hist, K, sm, tid);
   const uint32_t bmax = (uint32_t)sm.bin;
-  // B: the groups whose maximum reaches that bin
-  for (int g0 = 0; g0 < ng; g0 += kSelThreads) {
-    const int g = g0 + tid;
-    const bool q = g < ng && (IntKeys::key(__ldcg(gm + g)) >> kShift1) >= bmax;
-    const unsigned bal = __ballot_sync(0xffffffffu, q);
+  // B: the groups whose maximum reaches that bin, compacted with one shared
+  // atomic per warp (a warp scan of the threads' counts)
+  auto warp_slots = [&](int cnt, int *counter) {
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
     int base = 0;
-    if (lane == 0 && bal) base = atomicAdd(&sm.nq, __popc(bal));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    if (q) {
-      const int slot = base + __popc(bal & ((1u << lane) - 1u));
-      if (slot < kQGroups) sm.qg[slot] = g;
+    if (lane == 31 && incl > 0) base = atomicAdd(counter, incl);
+    return __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
+  };
+  for (int g0 = 0; g0 < ng; g0 += kSelThreads * 4) {
+    unsigned mq = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int g = g0 + j * kSelThreads + tid;
+      const int v = held ? vh[j] : (g < ng ? __ldcg(gm + g) : INT_MIN);
+      if (g < ng && (IntKeys::key(v) >> kShift1) >= bmax) mq |= 1u << j;
+    }
+    int slot = warp_slots(__popc(mq), &sm.nq);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if ((mq >> j) & 1u) {
+        if (slot < kQGroups) sm.qg[slot] = g0 + j * kSelThreads + tid;
+        ++slot;
+      }
     }
   }
   for (int i = tid; i < kHistBins; i += kSelThreads) sm.hist[i] = 0;
   __syncthreads();
   const int nq = sm.nq;
   if (nq > kQGroups || 4LL * nq * gsize > 3LL * n) return false;
-  // C: the qualifying groups' scores that reach the bin, as (~key, block)
+  // C: the qualifying groups' scores that reach the bin, as (~key, block),
+  // compacted as in B
   const int nv = nq * gsize / 4;
   for (int e0 = 0; e0 < nv; e0 += kSelThreads * 4) {
     int4 v[4];
@@ -575,21 +599,25 @@ __device__ bool select_by_group_maxima(const int32_t *sc, const int32_t *gm, int
         }
       }
     }
+    unsigned mc = 0;  // bit 4 j + c: score c of quad j reaches the bin
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int sv = c == 0 ? v[j].x : c == 1 ? v[j].y : c == 2 ? v[j].z : v[j].w;
-        const int row = rowv[j] + c;
-        const uint32_t k = IntKeys::key(sv);
-        const bool take = rowv[j] >= 0 && row < n && (k >> kShift1) >= bmax;
-        const unsigned bal = __ballot_sync(0xffffffffu, take);
-        int base = 0;
-        if (lane == 0 && bal) base = atomicAdd(&sm.nqc, __popc(bal));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (take) {
-          const int slot = base + __popc(bal & ((1u << lane) - 1u));
-          if (slot < kQCand) sm.qc[slot] = ((unsigned long long)(0xffffffffu - k) << 32) | (uint32_t)row;
+        if (rowv[j] >= 0 && rowv[j] + c < n && (IntKeys::key(sv) >> kShift1) >= bmax) mc |= 1u << (4 * j + c);
+      }
+    }
+    int slot = warp_slots(__popc(mc), &sm.nqc);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if ((mc >> (4 * j + c)) & 1u) {
+          const int sv = c == 0 ? v[j].x : c == 1 ? v[j].y : c == 2 ? v[j].z : v[j].w;
+          if (slot < kQCand)
+            sm.qc[slot] = ((unsigned long long)(0xffffffffu - IntKeys::key(sv)) << 32) | (uint32_t)(rowv[j] + c);
+          ++slot;
         }
       }
     }
@@ -714,10 +742,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
 // with 16-byte loads: an item is 8192/d rows of one request (8 KiB of low
 // bytes plus their high fields: 20 loads per lane, all in flight together).
 // Lane l owns dims 16*(l % LPR) .. +15 of its rows, which come in runs of 4
-// consecutive rows (one 16-byte load of the run's high-field words).  Plain
-// loads beat a shared-memory ring fed by bulk copies here (measured on this
-// GPU: ~7.0 vs ~3.9 TB/s on randomly permuted 4 KiB pages).  The block-table
-// entries of the next item are fetched while the current one computes.
+// consecutive rows (one 16-byte load of the run's high-field words).  The
+// block-table entries of the next item are fetched while the current one
+// computes.  The scan runs at the read rate of its access pattern: the same
+// loads with the arithmetic removed read randomly placed 2,560-byte pages
+// at 6.85-6.91 TB/s (7.07 TB/s when the pages are consecutive; 6.81-6.89
+// with the pages at 3,072- or 4,096-byte strides), and a per-warp ring of
+// cp.async.bulk page copies into shared memory at most 6.61 TB/s.
 
 constexpr int kScanThreads = 128;
 constexpr int kItemLoads = 16;  // 16-byte key loads per lane per item (8 KiB of low bytes per warp)
