@@ -111,11 +111,14 @@ struct FloatKeys {  // float32 scores (their bits) of the normalised indexer
 };
 
 // ------------------------------------------------------------ selection --
-// One CTA of kSelThreads threads per request.  The request's scores (written
-// by the scan kernel, L2-resident) are read with 16-byte loads issued in
-// batches of kSelBatch per thread, so many loads are in flight at once.
+// One CTA of NTH threads per request: 1,024 while the requests fit one wave
+// of one CTA per SM, else 512 (two CTAs per SM, half the waves; the host
+// picks).  The request's scores (written by the scan kernel, L2-resident)
+// are read with 16-byte loads issued in batches of kSelBatch per thread, so
+// many loads are in flight at once.
 
-constexpr int kSelThreads = 1024;
+constexpr int kSelThreads = 1024;       // the largest CTA
+constexpr int kSelThreadsPerSM = 1024;  // 64 registers per thread at most
 constexpr int kSelBatch = 8;  // int4 loads in flight per thread
 constexpr int kBitmapWords = 8192;  // requests of <= 262,144 blocks mark kept blocks in a bitmap
 
@@ -198,10 +201,11 @@ __device__ __forceinline__ void put_block(int32_t *out, int32_t *tok, int pos, i
 
 // Writes the set bits of bits[0 .. ceil(n/32)) as ascending indices:
 // exactly K bits are set.
+template <int NTH>
 __device__ void write_from_bits(const uint32_t *bits, int n, int K, int32_t *out, int32_t *tok,
                                 int p0, SelSmem &sm, int tid) {
   const int W = (n + 31) >> 5;
-  const int per = (W + kSelThreads - 1) / kSelThreads;
+  const int per = (W + NTH - 1) / NTH;
   const int w0 = min(W, tid * per), w1 = min(W, w0 + per);
   int cnt = 0;
   for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
@@ -217,10 +221,11 @@ __device__ void write_from_bits(const uint32_t *bits, int n, int K, int32_t *out
   }
 }
 
+template <int NTH>
 __device__ __forceinline__ void bitonic_sort_i32(int *a, int n_pow2, int tid) {
   for (int k = 2; k <= n_pow2; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < n_pow2; i += kSelThreads) {
+      for (int i = tid; i < n_pow2; i += NTH) {
         const int l = i ^ j;
         if (l > i) {
           const int x = a[i], y = a[l];
@@ -246,56 +251,56 @@ __device__ __forceinline__ int next_pow2(int x) {
 // 16-byte boundary (rows are 4-byte aligned; the row stride need not be a
 // multiple of 4): fq(index, int4) for each aligned quad, f(index, score) for
 // the scores before and after them.
-template <typename FQ, typename F>
+template <int NTH, typename FQ, typename F>
 __device__ __forceinline__ void for_each_score_q(const int32_t *sc, int n, int tid, FQ fq, F f) {
   const int head = min(n, (int)(((16u - (uint32_t)(reinterpret_cast<uintptr_t>(sc) & 15u)) & 15u) >> 2));
   if (tid < head) f(tid, __ldcg(sc + tid));
   const int4 *v4 = reinterpret_cast<const int4 *>(sc + head);
   const int nv = (n - head) >> 2;
-  for (int base = 0; base < nv; base += kSelThreads * kSelBatch) {
+  for (int base = 0; base < nv; base += NTH * kSelBatch) {
     int4 v[kSelBatch];
 #pragma unroll
     for (int j = 0; j < kSelBatch; ++j) {
-      const int i = base + j * kSelThreads + tid;
+      const int i = base + j * NTH + tid;
       v[j] = (i < nv) ? __ldcg(v4 + i) : make_int4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int j = 0; j < kSelBatch; ++j) {
-      const int i = base + j * kSelThreads + tid;
+      const int i = base + j * NTH + tid;
       if (i < nv) fq(head + 4 * i, v[j]);
     }
   }
-  for (int i = head + 4 * nv + tid; i < n; i += kSelThreads) f(i, __ldcg(sc + i));
+  for (int i = head + 4 * nv + tid; i < n; i += NTH) f(i, __ldcg(sc + i));
 }
 
 // Visits the scores of a row that may pass a filter: quads are loaded in
 // batches, reduced to one bit each by keep4(int4), and only the (rare)
 // flagged quads are read again and handed to f(index, score) element by
 // element; the scores before and after the aligned quads always go to f.
-template <typename K4, typename F>
+template <int NTH, typename K4, typename F>
 __device__ __forceinline__ void for_each_flagged_score(const int32_t *sc, int n, int tid, K4 keep4,
                                                        F f) {
   const int head = min(n, (int)(((16u - (uint32_t)(reinterpret_cast<uintptr_t>(sc) & 15u)) & 15u) >> 2));
   if (tid < head) f(tid, __ldcg(sc + tid));
   const int4 *v4 = reinterpret_cast<const int4 *>(sc + head);
   const int nv = (n - head) >> 2;
-  for (int base = 0; base < nv; base += kSelThreads * kSelBatch) {
+  for (int base = 0; base < nv; base += NTH * kSelBatch) {
     int4 v[kSelBatch];
 #pragma unroll
     for (int j = 0; j < kSelBatch; ++j) {
-      const int i = base + j * kSelThreads + tid;
+      const int i = base + j * NTH + tid;
       v[j] = (i < nv) ? __ldcg(v4 + i) : make_int4(INT_MIN, INT_MIN, INT_MIN, INT_MIN);
     }
     unsigned flags = 0;
 #pragma unroll
     for (int j = 0; j < kSelBatch; ++j) {
-      const int i = base + j * kSelThreads + tid;
+      const int i = base + j * NTH + tid;
       flags |= (i < nv && keep4(v[j]) ? 1u : 0u) << j;
     }
     while (flags) {
       const int j = __ffs(flags) - 1;
       flags &= flags - 1u;
-      const int i = base + j * kSelThreads + tid;
+      const int i = base + j * NTH + tid;
       const int4 w = __ldcg(v4 + i);
       const int e = head + 4 * i;
       f(e, w.x);
@@ -304,13 +309,13 @@ __device__ __forceinline__ void for_each_flagged_score(const int32_t *sc, int n,
       f(e + 3, w.w);
     }
   }
-  for (int i = head + 4 * nv + tid; i < n; i += kSelThreads) f(i, __ldcg(sc + i));
+  for (int i = head + 4 * nv + tid; i < n; i += NTH) f(i, __ldcg(sc + i));
 }
 
 // Applies f(index, score) to every score of a row.
-template <typename F>
+template <int NTH, typename F>
 __device__ __forceinline__ void for_each_score(const int32_t *sc, int n, int tid, F f) {
-  for_each_score_q(
+  for_each_score_q<NTH>(
       sc, n, tid,
       [&](int e, int4 v) {
         f(e, v.x);
@@ -324,8 +329,9 @@ __device__ __forceinline__ void for_each_score(const int32_t *sc, int n, int tid
 // Finds, in hist[0..nbins), the bin where the running count taken from the
 // top bin down first reaches `rank` (>= 1); writes it and the count strictly
 // above it to sm.bin / sm.above.  Ends with a barrier.
+template <int NTH>
 __device__ void find_rank_bin_desc(const int *hist, int rank, SelSmem &sm, int tid) {
-  constexpr int per = kHistBins / kSelThreads;
+  constexpr int per = kHistBins / NTH;
   int local = 0;
 #pragma unroll
   for (int k = 0; k < per; ++k) local += hist[kHistBins - 1 - (tid * per + k)];
@@ -358,7 +364,7 @@ __device__ void find_rank_bin_desc(const int *hist, int rank, SelSmem &sm, int t
 // radix passes over the score row establish the exact threshold key, then
 // (on a tie at the threshold) the largest kept index among the tied blocks,
 // then the kept set is gathered.
-template <typename KT>
+template <typename KT, int NTH>
 __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, int tid) {
   int *hist = sm.hist;
   constexpr int kShift1 = KT::kBits - 13;
@@ -368,9 +374,9 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
     const int nbits = min(kFbDigitBits, shift);
     const int nshift = shift - nbits;
     const int nbins = 1 << nbits;
-    for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+    for (int i = tid; i < kHistBins; i += NTH) hist[i] = 0;
     __syncthreads();
-    for_each_score(sc, n, tid, [&](int, int s) {
+    for_each_score<NTH>(sc, n, tid, [&](int, int s) {
       const uint32_t k = KT::key(s);
       if ((k >> shift) == prefix) atomicAdd(&hist[(k >> nshift) & (nbins - 1)], 1);
     });
@@ -396,7 +402,7 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
   if (tid == 0) sm.ncand = 0;
   __syncthreads();
   int myties = 0;
-  for_each_score(sc, n, tid, [&](int, int s) { myties += (KT::key(s) == tkey); });
+  for_each_score<NTH>(sc, n, tid, [&](int, int s) { myties += (KT::key(s) == tkey); });
   atomicAdd(&sm.ncand, myties);
   __syncthreads();
   int idx_limit = 0x7fffffff;
@@ -406,9 +412,9 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
     int before = 0;
     for (int pass = 0; pass < 3; ++pass) {
       const int sh = 16 - 8 * pass;
-      for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+      for (int i = tid; i < kHistBins; i += NTH) hist[i] = 0;
       __syncthreads();
-      for_each_score(sc, n, tid, [&](int i, int s) {
+      for_each_score<NTH>(sc, n, tid, [&](int i, int s) {
         if (KT::key(s) == tkey && ((uint32_t)i >> (sh + 8)) == ipre)
           atomicAdd(&hist[((uint32_t)i >> sh) & 255], 1);
       });
@@ -433,7 +439,7 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
   int *keep = sm.hist;
   if (tid == 0) sm.nkeep = 0;
   __syncthreads();
-  for_each_score(sc, n, tid, [&](int i, int s) {
+  for_each_score<NTH>(sc, n, tid, [&](int i, int s) {
     const uint32_t k = KT::key(s);
     if (k > tkey || (k == tkey && i <= idx_limit)) {
       const int slot = atomicAdd(&sm.nkeep, 1);
@@ -445,10 +451,11 @@ __device__ void select_fallback(const int32_t *sc, int n, int K, SelSmem &sm, in
 
 // Writes the K distinct kept indices in ascending order: by rank counting
 // for small K, by a bitonic sort otherwise.
+template <int NTH>
 __device__ void write_ascending(int *keep, int K, int32_t *out, int32_t *tok, int p0, SelSmem &sm,
                                 int tid) {
   if (K <= 1024) {
-    for (int i = tid; i < K; i += kSelThreads) {
+    for (int i = tid; i < K; i += NTH) {
       const int x = keep[i];
       int rank = 0;
       for (int j = 0; j < K; ++j) rank += (keep[j] < x);
@@ -457,25 +464,25 @@ __device__ void write_ascending(int *keep, int K, int32_t *out, int32_t *tok, in
     return;
   }
   const int kp2 = next_pow2(K);
-  for (int i = K + tid; i < kp2; i += kSelThreads) keep[i] = 0x7fffffff;
+  for (int i = K + tid; i < kp2; i += NTH) keep[i] = 0x7fffffff;
   __syncthreads();
-  bitonic_sort_i32(keep, kp2, tid);
-  for (int i = tid; i < K; i += kSelThreads) put_block(out, tok, i, keep[i], p0);
+  bitonic_sort_i32<NTH>(keep, kp2, tid);
+  for (int i = tid; i < K; i += NTH) put_block(out, tok, i, keep[i], p0);
 }
 
 // The two passes of the selection over a score row: a histogram of the
 // first digit, then a pass that keeps the blocks above the threshold bin
 // (bitmap when use_bits, else the list in sm.hist) and gathers the bin's
 // blocks.
-template <typename KT>
+template <typename KT, int NTH>
 __device__ void select_passes(const int32_t *sc, int n, int K, bool use_bits, SelSmem &sm,
                                int tid) {
   constexpr int kShift1 = KT::kBits - 13;
-  for_each_score(sc, n, tid, [&](int, int sv) {
+  for_each_score<NTH>(sc, n, tid, [&](int, int sv) {
     atomicAdd(&sm.hist[KT::key(sv) >> kShift1], 1);
   });
   __syncthreads();
-  find_rank_bin_desc(sm.hist, K, sm, tid);
+  find_rank_bin_desc<NTH>(sm.hist, K, sm, tid);
   const uint32_t b1 = (uint32_t)sm.bin;
   int *keep = sm.hist;
   auto visit = [&](int i, int sv) {
@@ -492,7 +499,7 @@ __device__ void select_passes(const int32_t *sc, int n, int K, bool use_bits, Se
     append_cand(d1 == b1, ((unsigned long long)(0xffffffffu - k) << 32) | (uint32_t)i, sm);
   };
   // a quad whose largest key is below the threshold bin is skipped whole
-  for_each_flagged_score(
+  for_each_flagged_score<NTH>(
       sc, n, tid, [&](int4 v) { return (KT::quad_max(v) >> kShift1) >= b1; }, visit);
   __syncthreads();
 }
@@ -514,6 +521,7 @@ __device__ void select_passes(const int32_t *sc, int n, int K, bool use_bits, Se
 // candidates, and the histogram / keep passes then run on them in shared
 // memory.  Reads ~16 KB of maxima and the qualifying groups' rows (~1/8 of
 // the row at 65,536 blocks) instead of the whole row twice.
+template <int NTH>
 __device__ bool select_by_group_maxima(const int32_t *sc, const int32_t *gm, int gsize, int n, int K,
                                        SelSmem &sm, int tid) {
   constexpr int kShift1 = IntKeys::kBits - 13;
@@ -521,25 +529,25 @@ __device__ bool select_by_group_maxima(const int32_t *sc, const int32_t *gm, int
   const int ng = (n + gsize - 1) / gsize;
   if (ng < 2 * K) return false;
   // A: histogram of the group maxima, the bin of the K-th largest.  Group
-  // g0 + j * kSelThreads + tid is this thread's j-th; with at most
-  // 4 * kSelThreads groups their maxima stay in registers for B.
-  const bool held = ng <= 4 * kSelThreads;
+  // g0 + j * NTH + tid is this thread's j-th; with at most
+  // 4 * NTH groups their maxima stay in registers for B.
+  const bool held = ng <= 4 * NTH;
   int vh[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
-  for (int g0 = 0; g0 < ng; g0 += kSelThreads * 4) {
+  for (int g0 = 0; g0 < ng; g0 += NTH * 4) {
     int v[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int g = g0 + j * kSelThreads + tid;
+      const int g = g0 + j * NTH + tid;
       v[j] = g < ng ? __ldcg(gm + g) : INT_MIN;
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      if (g0 + j * kSelThreads + tid < ng) atomicAdd(&sm.hist[IntKeys::key(v[j]) >> kShift1], 1);
+      if (g0 + j * NTH + tid < ng) atomicAdd(&sm.hist[IntKeys::key(v[j]) >> kShift1], 1);
       vh[j] = v[j];
     }
   }
   __syncthreads();
-  find_rank_bin_desc(sm.hist, K, sm, tid);
+  find_rank_bin_desc<NTH>(sm.hist, K, sm, tid);
   const uint32_t bmax = (uint32_t)sm.bin;
   // B: the groups whose maximum reaches that bin, compacted with one shared
   // atomic per warp (a warp scan of the threads' counts)
@@ -554,11 +562,11 @@ __device__ bool select_by_group_maxima(const int32_t *sc, const int32_t *gm, int
     if (lane == 31 && incl > 0) base = atomicAdd(counter, incl);
     return __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
   };
-  for (int g0 = 0; g0 < ng; g0 += kSelThreads * 4) {
+  for (int g0 = 0; g0 < ng; g0 += NTH * 4) {
     unsigned mq = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int g = g0 + j * kSelThreads + tid;
+      const int g = g0 + j * NTH + tid;
       const int v = held ? vh[j] : (g < ng ? __ldcg(gm + g) : INT_MIN);
       if (g < ng && (IntKeys::key(v) >> kShift1) >= bmax) mq |= 1u << j;
     }
@@ -566,24 +574,24 @@ __device__ bool select_by_group_maxima(const int32_t *sc, const int32_t *gm, int
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       if ((mq >> j) & 1u) {
-        if (slot < kQGroups) sm.qg[slot] = g0 + j * kSelThreads + tid;
+        if (slot < kQGroups) sm.qg[slot] = g0 + j * NTH + tid;
         ++slot;
       }
     }
   }
-  for (int i = tid; i < kHistBins; i += kSelThreads) sm.hist[i] = 0;
+  for (int i = tid; i < kHistBins; i += NTH) sm.hist[i] = 0;
   __syncthreads();
   const int nq = sm.nq;
   if (nq > kQGroups || 4LL * nq * gsize > 3LL * n) return false;
   // C: the qualifying groups' scores that reach the bin, as (~key, block),
   // compacted as in B
   const int nv = nq * gsize / 4;
-  for (int e0 = 0; e0 < nv; e0 += kSelThreads * 4) {
+  for (int e0 = 0; e0 < nv; e0 += NTH * 4) {
     int4 v[4];
     int rowv[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int e = e0 + j * kSelThreads + tid;
+      const int e = e0 + j * NTH + tid;
       rowv[j] = -1;
       v[j] = make_int4(INT_MIN, INT_MIN, INT_MIN, INT_MIN);
       if (e < nv) {
@@ -627,12 +635,12 @@ __device__ bool select_by_group_maxima(const int32_t *sc, const int32_t *gm, int
   if (nc > kQCand) return false;
   // D: histogram of the candidates, the threshold bin, keep the blocks above
   // it, gather the bin's blocks
-  for (int i = tid; i < nc; i += kSelThreads)
+  for (int i = tid; i < nc; i += NTH)
     atomicAdd(&sm.hist[(0xffffffffu - (uint32_t)(sm.qc[i] >> 32)) >> kShift1], 1);
   __syncthreads();
-  find_rank_bin_desc(sm.hist, K, sm, tid);
+  find_rank_bin_desc<NTH>(sm.hist, K, sm, tid);
   const uint32_t b1 = (uint32_t)sm.bin;
-  for (int i0 = 0; i0 < nc; i0 += kSelThreads) {
+  for (int i0 = 0; i0 < nc; i0 += NTH) {
     const int i = i0 + tid;
     bool take = false;
     unsigned long long x = 0;
@@ -650,8 +658,8 @@ __device__ bool select_by_group_maxima(const int32_t *sc, const int32_t *gm, int
 }
 
 // Selection kernel: grid = B, one request per CTA.
-template <typename KT>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
+template <typename KT, int NTH>
+__global__ void __launch_bounds__(NTH, kSelThreadsPerSM / NTH) select_kernel(Params p) {
   pdl_open();
   extern __shared__ uint8_t smem_raw[];
   SelSmem &sm = *reinterpret_cast<SelSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -664,7 +672,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
   int32_t *out = p.sel ? p.sel + (long long)r * K : nullptr;
   const int32_t *sc = p.scores + (long long)r * p.max_blocks;
   if (n <= K) {
-    for (int i = tid; i < K; i += kSelThreads) {
+    for (int i = tid; i < K; i += NTH) {
       if (i < n) {
         put_block(out, tok, i, i, p0);
       } else {
@@ -677,8 +685,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
   // kept blocks go to a bitmap when the request fits it, else to a list
   const bool use_bits = n <= kBitmapWords * 32;
   const int nwords = use_bits ? (n + 31) >> 5 : 0;
-  for (int i = tid; i < kHistBins; i += kSelThreads) sm.hist[i] = 0;
-  for (int i = tid; i < nwords; i += kSelThreads) sm.bits[i] = 0u;
+  for (int i = tid; i < kHistBins; i += NTH) sm.hist[i] = 0;
+  for (int i = tid; i < nwords; i += NTH) sm.bits[i] = 0u;
   if (tid == 0) {
     sm.nkeep = 0;
     sm.ncand = 0;
@@ -689,11 +697,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
   bool done = false;
   if constexpr (KT::kBits == IntKeys::kBits) {
     if (p.gmax && use_bits) {
-      done = select_by_group_maxima(sc, p.gmax + (long long)r * ((p.max_blocks + p.gsize - 1) / p.gsize),
+      done = select_by_group_maxima<NTH>(sc, p.gmax + (long long)r * ((p.max_blocks + p.gsize - 1) / p.gsize),
                                     p.gsize, n, K, sm, tid);
       if (!done) {  // start over with the two full passes
-        for (int i = tid; i < kHistBins; i += kSelThreads) sm.hist[i] = 0;
-        for (int i = tid; i < nwords; i += kSelThreads) sm.bits[i] = 0u;
+        for (int i = tid; i < kHistBins; i += NTH) sm.hist[i] = 0;
+        for (int i = tid; i < nwords; i += NTH) sm.bits[i] = 0u;
         if (tid == 0) {
           sm.nkeep = 0;
           sm.ncand = 0;
@@ -702,7 +710,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
       }
     }
   }
-  if (!done) select_passes<KT>(sc, n, K, use_bits, sm, tid);
+  if (!done) select_passes<KT, NTH>(sc, n, K, use_bits, sm, tid);
   int *keep = sm.hist;
   const int above = sm.above;
   const int ncand = sm.ncand;
@@ -713,7 +721,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
     // shared atomics on the ranks, measured slower: 19.7 against 17.5 us per
     // launch, the ~50 rank counters contended.)
     const int need = K - above;
-    for (int i = tid; i < ncand; i += kSelThreads) {
+    for (int i = tid; i < ncand; i += NTH) {
       const unsigned long long x = sm.cand[i];
       int rank = 0;
       for (int j = 0; j < ncand; ++j) rank += (sm.cand[j] < x);
@@ -725,16 +733,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params p) {
     }
     __syncthreads();
   } else {
-    select_fallback<KT>(sc, n, K, sm, tid);  // the kept list, in sm.hist
+    select_fallback<KT, NTH>(sc, n, K, sm, tid);  // the kept list, in sm.hist
     if (use_bits) {
-      for (int i = tid; i < nwords; i += kSelThreads) sm.bits[i] = 0u;
+      for (int i = tid; i < nwords; i += NTH) sm.bits[i] = 0u;
       __syncthreads();
-      for (int i = tid; i < K; i += kSelThreads) atomicOr(&sm.bits[keep[i] >> 5], 1u << (keep[i] & 31));
+      for (int i = tid; i < K; i += NTH) atomicOr(&sm.bits[keep[i] >> 5], 1u << (keep[i] & 31));
       __syncthreads();
     }
   }
-  if (use_bits) write_from_bits(sm.bits, n, K, out, tok, p0, sm, tid);
-  else write_ascending(keep, K, out, tok, p0, sm, tid);
+  if (use_bits) write_from_bits<NTH>(sm.bits, n, K, out, tok, p0, sm, tid);
+  else write_ascending<NTH>(keep, K, out, tok, p0, sm, tid);
 }
 
 // ------------------------------------------------------------- the scan --

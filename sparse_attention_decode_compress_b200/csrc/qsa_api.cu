@@ -139,19 +139,43 @@ std::mutex g_mutex;
 // ------------------------------------------------------------------ topk --
 size_t select_smem() { return sizeof(qsa::topk::SelSmem) + 128; }
 
+template <typename KT, int NTH>
+qsa_status launch_select_nth(const qsa::topk::Params &p, cudaStream_t stream) {
+  static bool done[kMaxDevices] = {false};
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (prepare_kernel(qsa::topk::select_kernel<KT, NTH>, select_smem(), done) != cudaSuccess)
+      return QSA_ERR_CUDA;
+  }
+  return launch(true, qsa::topk::select_kernel<KT, NTH>, dim3((unsigned)p.B), dim3(NTH), select_smem(),
+                stream, p);
+}
+
+// The selection, one CTA per request: 1,024 threads, or 512 threads (two
+// CTAs per SM: registers and shared memory allow two) for more requests
+// than SMs of at most 32,768 blocks, which then take half the waves.  Long
+// requests keep 1,024 threads: on the mixed fp8 batch (256 requests of up
+// to 262,144 blocks) one wave of 512-thread CTAs took 46 us, two waves of
+// 1,024-thread CTAs 39 us; the sparse prefill's 4,096 tokens of ~8,192
+// blocks took 156 against 245 us.
+constexpr int kSelHalfMaxBlocks = 32768;
+template <typename KT>
+qsa_status launch_select(const qsa::topk::Params &p, cudaStream_t stream) {
+  if (p.B > sm_count(current_device()) && p.max_blocks <= kSelHalfMaxBlocks)
+    return launch_select_nth<KT, 512>(p, stream);
+  return launch_select_nth<KT, qsa::topk::kSelThreads>(p, stream);
+}
+
 // Scan (persistent grid, scores to the buffer) then selection (one CTA per
 // request), back to back on the caller's stream.
 template <int DI, int BPPC>
 qsa_status launch_index_topk(const qsa::topk::Params &p, cudaStream_t stream) {
   using namespace qsa::topk;
-  static bool done_sel[kMaxDevices] = {false};
   static int blocks_per_sm[kMaxDevices] = {0};
   auto kernel = index_scan_kernel<DI, BPPC>;
   const int dev = current_device();
   {
     std::lock_guard<std::mutex> lk(g_mutex);
-    if (prepare_kernel(select_kernel<IntKeys>, select_smem(), done_sel) != cudaSuccess)
-      return QSA_ERR_CUDA;
     if (dev >= 0 && dev < kMaxDevices && !blocks_per_sm[dev]) {
       int n = 0;
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kScanThreads, 0) != cudaSuccess)
@@ -163,7 +187,7 @@ qsa_status launch_index_topk(const qsa::topk::Params &p, cudaStream_t stream) {
   const int grid = bps * sm_count(dev);
   qsa_status st = launch(true, kernel, dim3(grid), dim3(kScanThreads), 0, stream, p);
   if (st != QSA_OK) return st;
-  return launch(true, select_kernel<IntKeys>, dim3(p.B), dim3(kSelThreads), select_smem(), stream, p);
+  return launch_select<IntKeys>(p, stream);
 }
 
 // Scan instance for the indexer dim and page geometry: constant page
@@ -728,14 +752,11 @@ namespace {
 template <int DI>
 qsa_status launch_index_topk_norm(const qsa::norm::ScanParams &sp, cudaStream_t stream) {
   using namespace qsa::topk;
-  static bool done_sel[kMaxDevices] = {false};
   static int blocks_per_sm[kMaxDevices] = {0};
   auto kernel = qsa::norm::index_scan_norm_kernel<DI>;
   const int dev = current_device();
   {
     std::lock_guard<std::mutex> lk(g_mutex);
-    if (prepare_kernel(select_kernel<FloatKeys>, select_smem(), done_sel) != cudaSuccess)
-      return QSA_ERR_CUDA;
     if (dev >= 0 && dev < kMaxDevices && !blocks_per_sm[dev]) {
       int n = 0;
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, qsa::norm::kScanThreads, 0) !=
@@ -748,8 +769,7 @@ qsa_status launch_index_topk_norm(const qsa::norm::ScanParams &sp, cudaStream_t 
   qsa_status st = launch(true, kernel, dim3(bps * sm_count(dev)), dim3(qsa::norm::kScanThreads), 0,
                          stream, sp);
   if (st != QSA_OK) return st;
-  return launch(true, select_kernel<FloatKeys>, dim3(sp.p.B), dim3(kSelThreads), select_smem(),
-                stream, sp.p);
+  return launch_select<FloatKeys>(sp.p, stream);
 }
 
 bool norm_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
@@ -950,13 +970,6 @@ qsa_status qsa_sparse_prefill(const qsa_cache *cache, int32_t B, int32_t n_token
               dim3(256), 0, s, pp);
   if (st != QSA_OK) return st;
   // 3. per-token selection over blocks 0 .. floor(p/4)
-  {
-    static bool done_sel[kMaxDevices] = {false};
-    std::lock_guard<std::mutex> lk(g_mutex);
-    if (prepare_kernel(qsa::topk::select_kernel<qsa::topk::IntKeys>, select_smem(), done_sel) !=
-        cudaSuccess)
-      return QSA_ERR_CUDA;
-  }
   qsa::topk::Params tp;
   tp.c = to_dev(cache);
   tp.B = n_tokens;
@@ -967,8 +980,7 @@ qsa_status qsa_sparse_prefill(const qsa_cache *cache, int32_t B, int32_t n_token
   tp.topk = topk;
   tp.sel = sel;
   tp.scores = scores;
-  st = launch(true, qsa::topk::select_kernel<qsa::topk::IntKeys>, dim3((unsigned)n_tokens),
-              dim3(qsa::topk::kSelThreads), select_smem(), s, tp);
+  st = launch_select<qsa::topk::IntKeys>(tp, s);
   if (st != QSA_OK) return st;
   // 4. attention of every token over its kept tokens (one split: o, lse)
   return sparse_decode_call(cache, n_tokens, 1, Hq, q, q_dtype, tok_len, sel, topk, sm_scale, 1, 0,

@@ -294,12 +294,14 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_streamk_kernel(SKPar
 // o = 0, lse = -inf).  With `o` set, the row's splits are then merged into
 // o / lse with the operations of merge_row (qsa_lse_merge), on the values
 // just computed, so the result has the same bits as qsa_lse_merge of o_part.
-// The (split, slot) pairs of the row are flattened across the lanes: a
-// first pass over their lse takes each split's maximum, a second weighs
-// every slot by exp(lse - maximum) (lane-parallel) and sums the weights and
-// the weighted rows (a float4 slice per lane, 16 slot rows loaded
-// together) in slot order, so a split's bits do not depend on the lanes its
-// slots land on (which depend on the splits a call computes).  (A running maximum with a rescale per
+// The (split, slot) pairs of the row are flattened across the lanes: each
+// split's maximum lse is taken first, then every slot is weighed by
+// exp(lse - maximum) (lane-parallel) and the weights and the weighted rows
+// (a float4 slice per lane, 16 slot rows loaded together) are summed in
+// slot order, so a split's bits do not depend on the lanes its slots land
+// on (which depend on the splits a call computes).  Up to 16 slots per row
+// take one round of loads (lse and rows together); more take a pass over
+// the lse for the maxima and a second over lse and rows.  (A running maximum with a rescale per
 // slot, serial over the slots, cost ~60 instructions per slot: 15 us per
 // launch at batch 16 with ~32 slots per split, 8.6 us at batch 128.)
 constexpr int kSKMergeThreads = 128;
@@ -356,15 +358,17 @@ __global__ void __launch_bounds__(kSKMergeThreads) streamk_merge_kernel(SKParams
     }
     slot = (P * p.S + p.s_lo + max(si, 0)) * sk.K + kk;
   };
-  // pass 1: each split's maximum lse
   float mxs[NSMAX];
+  float4 os[NSMAX];
+  float dens[NSMAX];
 #pragma unroll
-  for (int i = 0; i < NSMAX; ++i) mxs[i] = -INFINITY;
-  for (int base = 0; base < total; base += 32) {
-    int si;
-    long long slot;
-    locate(base + lane, si, slot);
-    const float lv = (si >= 0) ? __ldcg(sk.sk_lse + slot * p.M + m) : -INFINITY;
+  for (int i = 0; i < NSMAX; ++i) {
+    mxs[i] = -INFINITY;
+    os[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    dens[i] = 0.f;
+  }
+  // the running maximum of each split over the lanes' slots
+  auto split_max = [&](int si, float lv) {
 #pragma unroll
     for (int i = 0; i < NSMAX; ++i) {
       if (i >= ns) break;
@@ -373,51 +377,75 @@ __global__ void __launch_bounds__(kSKMergeThreads) streamk_merge_kernel(SKParams
       for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
       mxs[i] = fmaxf(mxs[i], x);
     }
-  }
-  // pass 2: weights, their sums and the weighted rows
-  float4 os[NSMAX];
-  float dens[NSMAX];
-#pragma unroll
-  for (int i = 0; i < NSMAX; ++i) {
-    os[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    dens[i] = 0.f;
-  }
-  for (int base = 0; base < total; base += 32) {
-    int si;
-    long long slot;
-    locate(base + lane, si, slot);
-    const float lv = (si >= 0) ? __ldcg(sk.sk_lse + slot * p.M + m) : -INFINITY;
+  };
+  // exp(lse - its split's maximum), 0 for an empty segment
+  auto weight = [&](int si, float lv) {
     float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < NSMAX; ++i)
       if (i == si) mx = mxs[i];
-    const float wgt = (lv == -INFINITY) ? 0.f : __expf(lv - mx);
-    const int nb = min(32, total - base);
-    for (int sub = 0; sub < nb; sub += kSKMergeSlots) {
-      float4 v[kSKMergeSlots];
-      const int nround = min(kSKMergeSlots, nb - sub);
+    return (lv == -INFINITY) ? 0.f : __expf(lv - mx);
+  };
+  // the rows of slots sub .. sub + nround - 1 (held by those lanes), loaded together
+  auto load_rows = [&](float4 (&v)[kSKMergeSlots], long long slot, int sub, int nround) {
 #pragma unroll
-      for (int j = 0; j < kSKMergeSlots; ++j) {
-        const long long sj = __shfl_sync(0xffffffffu, slot, sub + j);
-        v[j] = (j < nround && d < D)
-                   ? __ldcg(reinterpret_cast<const float4 *>(sk.sk_o + (sj * p.M + m) * D + d))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < kSKMergeSlots; ++j) {
+      const long long sj = __shfl_sync(0xffffffffu, slot, sub + j);
+      v[j] = (j < nround && d < D)
+                 ? __ldcg(reinterpret_cast<const float4 *>(sk.sk_o + (sj * p.M + m) * D + d))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  // weights and weighted rows added in slot order
+  auto accumulate = [&](const float4 (&v)[kSKMergeSlots], int si, float wgt, int sub, int nround) {
+#pragma unroll
+    for (int j = 0; j < kSKMergeSlots; ++j) {
+      if (j >= nround) break;
+      const int i = __shfl_sync(0xffffffffu, si, sub + j);
+      const float w = __shfl_sync(0xffffffffu, wgt, sub + j);
+      if (w == 0.f) continue;  // an empty segment (or an unwritten slot) adds nothing
+#pragma unroll
+      for (int q = 0; q < NSMAX; ++q) {
+        if (q != i) continue;
+        dens[q] += w;
+        os[q].x = __fmaf_rn(w, v[j].x, os[q].x);
+        os[q].y = __fmaf_rn(w, v[j].y, os[q].y);
+        os[q].z = __fmaf_rn(w, v[j].z, os[q].z);
+        os[q].w = __fmaf_rn(w, v[j].w, os[q].w);
       }
-#pragma unroll
-      for (int j = 0; j < kSKMergeSlots; ++j) {
-        if (j >= nround) break;
-        const int i = __shfl_sync(0xffffffffu, si, sub + j);
-        const float w = __shfl_sync(0xffffffffu, wgt, sub + j);
-        if (w == 0.f) continue;  // an empty segment (or an unwritten slot) adds nothing
-#pragma unroll
-        for (int q = 0; q < NSMAX; ++q) {
-          if (q != i) continue;
-          dens[q] += w;
-          os[q].x = __fmaf_rn(w, v[j].x, os[q].x);
-          os[q].y = __fmaf_rn(w, v[j].y, os[q].y);
-          os[q].z = __fmaf_rn(w, v[j].z, os[q].z);
-          os[q].w = __fmaf_rn(w, v[j].w, os[q].w);
-        }
+    }
+  };
+  if (total <= kSKMergeSlots) {
+    // one round: the slots' lse and rows loaded together
+    int si;
+    long long slot;
+    locate(lane, si, slot);
+    const float lv = (si >= 0) ? __ldcg(sk.sk_lse + slot * p.M + m) : -INFINITY;
+    float4 v[kSKMergeSlots];
+    load_rows(v, slot, 0, total);
+    split_max(si, lv);
+    accumulate(v, si, weight(si, lv), 0, total);
+  } else {
+    // pass 1: each split's maximum lse
+    for (int base = 0; base < total; base += 32) {
+      int si;
+      long long slot;
+      locate(base + lane, si, slot);
+      split_max(si, (si >= 0) ? __ldcg(sk.sk_lse + slot * p.M + m) : -INFINITY);
+    }
+    // pass 2: the weights and the weighted rows
+    for (int base = 0; base < total; base += 32) {
+      int si;
+      long long slot;
+      locate(base + lane, si, slot);
+      const float lv = (si >= 0) ? __ldcg(sk.sk_lse + slot * p.M + m) : -INFINITY;
+      const float wgt = weight(si, lv);
+      const int nb = min(32, total - base);
+      for (int sub = 0; sub < nb; sub += kSKMergeSlots) {
+        float4 v[kSKMergeSlots];
+        const int nround = min(kSKMergeSlots, nb - sub);
+        load_rows(v, slot, sub, nround);
+        accumulate(v, si, wgt, sub, nround);
       }
     }
   }

@@ -86,3 +86,19 @@ def test_beyond_the_bitmap_with_every_score_tied():
     assert step.sel[0].cpu().tolist() == list(range(2048))
     for r in range(b.w.batch):
         H.check_request(b, step, cache, r, 2)
+
+
+# More requests than SMs, none longer than 32,768 blocks, take the selection
+# in CTAs of 512 threads, two per SM: the group maxima (from 16,384 blocks at
+# topk 512), the two passes, and rows shorter than topk, at half the threads.
+@pytest.mark.parametrize("topk", [512, 2048])
+def test_more_requests_than_sms_take_the_half_size_selection(topk):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    lens = [131072, 100001, 70001, 65537, 33000] + [4099 + 37 * i for i in range(sms)]
+    w = replace(WORKLOADS["b128_256k"], planted=8, topk=topk)
+    b = make_batch(w, "cuda", ctx_lens=lens, seed=41)
+    step, cache = H.run_gpu(b, 2)
+    assert H.check_index_every_request(b, step.sel, step.scores) == len(lens)
+    for r in (0, 1, 2, 3, 4, len(lens) - 1):
+        H.check_request(b, step, cache, r, 2)
+    H.check_properties(b, step)
