@@ -19,6 +19,7 @@
 #include "sparse_decode_warp.cuh"
 #include "sparse_decode_group.cuh"
 #include "sparse_decode_streamk.cuh"
+#include "sparse_decode_streamk_group.cuh"
 #include "lse_merge.cuh"
 
 namespace {
@@ -358,15 +359,23 @@ SKLayout sk_layout(int B, int T, int Hq, int Hkv, int topk, int S, int D) {
   return l;
 }
 
-template <int D>
-qsa_status launch_decode_streamk(const qsa::dec::Params &p, float *o, float *lse, void *workspace,
-                                 cudaStream_t stream) {
-  constexpr int NW = kDecWarps;
-  constexpr int NS = kDecStages;
+// Stream-K decode of bf16 caches and its merge.  GW = 1: one warp per
+// worker (at most 8 query rows per kv head); GW = 2..4: groups of GW warps,
+// one per 8-row tile, share a worker's ring.
+template <int D, int GW>
+qsa_status launch_decode_streamk_gw(const qsa::dec::Params &p, float *o, float *lse, void *workspace,
+                                    cudaStream_t stream) {
+  constexpr int NW = GW == 1 ? kDecWarps : 16 / GW * GW;
+  constexpr int NS = GW == 1 ? kDecStages : GW;
   static bool done[kMaxDevices] = {false};
   static int blocks_per_sm[kMaxDevices] = {0};
-  auto kernel = qsa::dec::sparse_decode_streamk_kernel<D, NW, NS>;
-  const size_t smem = sizeof(qsa::dec::WarpSmem<D, false, NW, NS>) + 128;
+  auto kernel = []() {
+    if constexpr (GW == 1) return qsa::dec::sparse_decode_streamk_kernel<D, NW, NS>;
+    else return qsa::dec::sparse_decode_streamk_group_kernel<D, NW, NS, GW>;
+  }();
+  const size_t smem = (GW == 1 ? sizeof(qsa::dec::WarpSmem<D, false, NW, NS>)
+                               : sizeof(qsa::dec::SKGroupSmem<D, NW, NS, GW>)) +
+                      128;
   const int dev = current_device();
   {
     std::lock_guard<std::mutex> lk(g_mutex);
@@ -379,16 +388,17 @@ qsa_status launch_decode_streamk(const qsa::dec::Params &p, float *o, float *lse
     }
   }
   const int bps = (dev >= 0 && dev < kMaxDevices) ? blocks_per_sm[dev] : 1;
+  constexpr int per_cta = NW / GW;  // workers per CTA
   qsa::dec::SKParams sk;
   sk.p = p;
-  sk.p.chunk = 1 << 20;  // the plan's chunk count is not used by this kernel
+  sk.p.chunk = 1 << 20;  // the plan's chunk count is not used by these kernels
   const long long pairs = (long long)p.B * p.c.num_kv_heads;
   sk.E = sk_entries(p.topk, p.T);
   sk.X = pairs * sk.E;
   sk.K = sk_slots(pairs, sk.E);
-  // one wave of resident CTAs at most; warps past W return at once
-  sk.W = (int)sk_warps(sk.X, (long long)bps * sm_count(dev) * NW);
-  const long long ctas = (sk.W + NW - 1) / NW;
+  // one wave of resident CTAs at most; workers past W return at once
+  sk.W = (int)sk_warps(sk.X, (long long)bps * sm_count(dev) * per_cta);
+  const long long ctas = (sk.W + per_cta - 1) / per_cta;
   const SKLayout lay = sk_layout(p.B, p.T, p.Hq, p.c.num_kv_heads, p.topk, p.S, D);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   sk.sk_ebound = reinterpret_cast<int32_t *>(ws + lay.ebound);
@@ -404,6 +414,17 @@ qsa_status launch_decode_streamk(const qsa::dec::Params &p, float *o, float *lse
   auto merge = (p.s_hi - p.s_lo <= 4) ? qsa::dec::streamk_merge_kernel<D, 4>
                                       : qsa::dec::streamk_merge_kernel<D, qsa::dec::kMaxSplits>;
   return launch(true, merge, dim3((unsigned)grid), dim3(qsa::dec::kSKMergeThreads), 0, stream, sk);
+}
+
+template <int D>
+qsa_status launch_decode_streamk(const qsa::dec::Params &p, float *o, float *lse, void *workspace,
+                                 cudaStream_t stream) {
+  switch ((p.M + 7) / 8) {  // 8-row tiles of the query rows
+    case 1: return launch_decode_streamk_gw<D, 1>(p, o, lse, workspace, stream);
+    case 2: return launch_decode_streamk_gw<D, 2>(p, o, lse, workspace, stream);
+    case 3: return launch_decode_streamk_gw<D, 3>(p, o, lse, workspace, stream);
+    default: return launch_decode_streamk_gw<D, 4>(p, o, lse, workspace, stream);
+  }
 }
 
 template <int D, bool FP8>
@@ -602,9 +623,9 @@ qsa_status sparse_decode_call(const qsa_cache *cache, int32_t B, int32_t T, int3
   if (B > 65535 || Hkv > 65535) return QSA_ERR_UNSUPPORTED;
   // cache rows are indexed with 32-bit integers
   if ((long long)cache->num_pages * cache->page_size * Hkv > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
-  // bf16 caches with at most 8 query rows per kv head take the stream-K
-  // decode; the rest the chunked decode with its ticket header
-  const bool streamk = cache->kv_dtype == QSA_BF16 && G * T <= 8;
+  // bf16 caches take the stream-K decode (one warp, or a warp group, per
+  // worker); fp8 and fp32 the chunked decode with its ticket header
+  const bool streamk = cache->kv_dtype == QSA_BF16;
   if (!streamk && (size_t)B * Hkv * num_splits * sizeof(int32_t) >
                       kTicketBytes - qsa::dec::kCounterInts * sizeof(int32_t))
     return QSA_ERR_UNSUPPORTED;

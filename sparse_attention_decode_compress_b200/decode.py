@@ -43,11 +43,9 @@ class QSADecodeStep:
     @property
     def kernels_per_step(self) -> int:
         """Kernels one step launches: append, scan, select, then the decode
-        and its merge; the chunked decode (float32 or fp8 caches, or more
-        than 8 query rows per kv head) adds the kernel that zeroes its
-        workspace header."""
-        G = self.Hq // self.cache.k_cache.shape[2]
-        chunked = self.cache.k_cache.dtype != torch.bfloat16 or G * self.T > 8
+        and its merge; the chunked decode (float32 or fp8 caches) adds the
+        kernel that zeroes its workspace header."""
+        chunked = self.cache.k_cache.dtype != torch.bfloat16
         return 6 if chunked else 5
 
 
