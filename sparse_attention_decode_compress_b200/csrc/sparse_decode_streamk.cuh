@@ -89,30 +89,6 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_streamk_kernel(SKPar
     const int e_lo = (int)(x - P * sk.E);
     const int e_hi = (int)(min(x_end, (P + 1) * sk.E) - P * sk.E);
     x = P * sk.E + e_hi;
-    if ((int)P != q_pair) {
-      // Q as B fragments (as sparse_decode_warp_kernel), issued before the
-      // plan so the loads overlap it; rows >= M are zero
-      const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        const int m = 8 * j + gq;
-        const bool ok = m < p.M;
-        const __nv_bfloat16 *qrow =
-            qg + (((long long)r * p.T + (ok ? m / p.G : 0)) * p.Hq + g * p.G + (ok ? m % p.G : 0)) * D;
-#pragma unroll
-        for (int kk = 0; kk < MD; ++kk) {
-          qb[j][kk][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq) : 0u;
-          qb[j][kk][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq + 8) : 0u;
-        }
-        csc[j][0] = csc[j][1] = p.scale_log2;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int mm = 8 * j + 2 * cq + e;
-          tcol[j][e] = mm < p.M ? mm / p.G : -1;
-        }
-      }
-      q_pair = (int)P;
-    }
     if (r != planned_r) {
       // the selection row is stashed in the ring's last slot (idle until
       // its stage): only the metadata fill right after the plan reads it,
@@ -156,6 +132,32 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_streamk_kernel(SKPar
         for (int s0 = 0; s0 < NS - 1; ++s0) {
           if (s0 < nst) issue_stage_warp<D, false>(p, W, s0, s0, lane);
           cp_async_commit();
+        }
+        if ((int)P != q_pair) {
+          // Q as B fragments (as sparse_decode_warp_kernel), rows >= M zero,
+          // loaded behind the first stages: the warp barriers of the plan
+          // and the metadata fill wait for the warp's loads in flight, so Q
+          // issued before them held the prologue up by its own latency
+          const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            const int m = 8 * j + gq;
+            const bool ok = m < p.M;
+            const __nv_bfloat16 *qrow =
+                qg + (((long long)r * p.T + (ok ? m / p.G : 0)) * p.Hq + g * p.G + (ok ? m % p.G : 0)) * D;
+#pragma unroll
+            for (int kk = 0; kk < MD; ++kk) {
+              qb[j][kk][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq) : 0u;
+              qb[j][kk][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq + 8) : 0u;
+            }
+            csc[j][0] = csc[j][1] = p.scale_log2;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int mm = 8 * j + 2 * cq + e;
+              tcol[j][e] = mm < p.M ? mm / p.G : -1;
+            }
+          }
+          q_pair = (int)P;
         }
         for (int st = 0; st < nst; ++st) {
           {

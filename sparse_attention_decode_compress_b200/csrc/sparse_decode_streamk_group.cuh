@@ -112,21 +112,6 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_streamk_group_kernel
     const int e_lo = (int)(x - P * sk.E);
     const int e_hi = (int)(min(x_end, (P + 1) * sk.E) - P * sk.E);
     x = P * sk.E + e_hi;
-    if (P != q_pair) {
-      // Q B-fragments of this warp's tile (rows m = 8 * wig + gq), issued
-      // before the plan so the loads overlap it
-      const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
-      const int m = 8 * wig + gq;
-      const bool ok = m < p.M;
-      const __nv_bfloat16 *qrow =
-          qg + (((long long)r * p.T + (ok ? m / p.G : 0)) * p.Hq + g * p.G + (ok ? m % p.G : 0)) * D;
-#pragma unroll
-      for (int kk = 0; kk < MD; ++kk) {
-        qb[kk][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq) : 0u;
-        qb[kk][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq + 8) : 0u;
-      }
-      q_pair = P;
-    }
     if (r != planned_r) {
       // the ring is idle once every warp has drained it; the selection row
       // goes to its last slot, read only by the metadata fill right after
@@ -163,6 +148,22 @@ __global__ void __launch_bounds__(NW * 32, 1) sparse_decode_streamk_group_kernel
         for (int s0 = 0; s0 < NS - 1; ++s0) {
           if (s0 < nst) issue_stage_group<D, false, GW>(p, W, s0, s0, tig);
           cp_async_commit();
+        }
+        if (P != q_pair) {
+          // Q B-fragments of this warp's tile (rows m = 8 * wig + gq),
+          // loaded behind the first stages (the barriers of the plan and the
+          // metadata fill wait for the loads in flight)
+          const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
+          const int m = 8 * wig + gq;
+          const bool ok = m < p.M;
+          const __nv_bfloat16 *qrow =
+              qg + (((long long)r * p.T + (ok ? m / p.G : 0)) * p.Hq + g * p.G + (ok ? m % p.G : 0)) * D;
+#pragma unroll
+          for (int kk = 0; kk < MD; ++kk) {
+            qb[kk][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq) : 0u;
+            qb[kk][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * cq + 8) : 0u;
+          }
+          q_pair = P;
         }
         for (int st = 0; st < nst; ++st) {
           cp_async_wait<NS - 2>();  // this thread's share of stage st has landed
