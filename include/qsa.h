@@ -257,11 +257,13 @@ size_t qsa_sparse_decode_workspace_bytes(int32_t B, int32_t T, int32_t Hq, int32
  *   o_part   [S, B, T, Hq, D] float32 output
  *   lse_part [S, B, T, Hq] float32 output (natural log)
  *   workspace  >= qsa_sparse_decode_workspace_bytes(...), 16-byte aligned,
- *            any contents: its header holds the work counter and the
+ *            any contents.  BF16 caches (the stream-K decode) keep the
+ *            requests' split boundaries and the workers' partials there,
+ *            all written before they are read.  FP8 and F32 caches (the
+ *            chunked decode) keep a header with a work counter and
  *            per-split tickets, which the call zeroes itself (a one-CTA
- *            kernel ahead of the decode kernel); the rest holds chunk
- *            partials.  Calls that overlap on the GPU need separate
- *            workspaces.
+ *            kernel ahead of the decode kernel), then the chunk partials.
+ *            Calls that overlap on the GPU need separate workspaces.
  * Errors: QSA_ERR_INVALID_ARG / QSA_ERR_UNSUPPORTED on the host
  * (QSA_ERR_UNSUPPORTED also when num_pages * page_size * Hkv exceeds
  * 2^31 - 1 cache rows); page or position violations -> QSA_ERR_BOUNDS on the

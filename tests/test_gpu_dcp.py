@@ -22,9 +22,13 @@ def _cuda_and_cleanup():
     torch.cuda.empty_cache()
 
 
+# short requests (fewer pages than splits: some of their splits are empty,
+# so a rank may see nothing of them) next to long ones
 @pytest.mark.parametrize("name,lens,S", [("b32_32k", [9000, 12345, 4099], 2),
+                                         ("b32_32k", [100, 9000, 70, 3001], 4),
                                          ("b128_256k", [40000, 30001], 4),
                                          ("mtp_verify", [16384 + 3, 9001], 2),
+                                         ("mtp_verify", [131, 5003, 70], 4),
                                          ("mixed_fp8", [4096, 30007], 4)])
 def test_split_ranges_match_full_decode(name, lens, S):
     b = make_batch(WORKLOADS[name], "cuda", ctx_lens=lens, seed=8)
