@@ -784,7 +784,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     line = run_ours(args, rank, world, local_rank)
     if rank == 0 and line is not None:
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:  # the host baseline: one GPU runs only
             from workloads.qsa_inputs import WORKLOADS
             w = WORKLOADS[args.workload]
             one = time_oracle(w, args.splits, args.cpu_queries)
