@@ -188,3 +188,22 @@ def test_norm_indexer_ties_take_the_lowest_blocks():
     assert got["sel"][0].cpu().tolist() == list(range(512))
     assert got["sel"][1].cpu().tolist() == list(range(512))
     _check(b, ni, got, 2)
+
+
+# More requests than SMs, each at most 32,768 blocks: the selection on float
+# keys runs in CTAs of 512 threads, two per SM (its two passes, and the exact
+# fallback when every score ties).
+@pytest.mark.parametrize("ties", [False, True])
+def test_norm_indexer_more_requests_than_sms(ties):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    lens = [32768, 20001] + [2100 + 61 * i for i in range(sms)]
+    w = replace(WORKLOADS["b32_32k"], planted=0 if ties else 8)
+    b = make_batch(w, "cuda", ctx_lens=lens, seed=64)
+    ni = norm_indexer_inputs(b, seed=64)
+    if ties:
+        ni["k"][:] = ni["k"][0].clone()
+    got = _run(b, ni, 2)
+    if ties:
+        for r in range(len(lens)):
+            assert got["sel"][r].cpu().tolist() == list(range(512)), r
+    _check(b, ni, got, 2)
