@@ -125,8 +125,9 @@ def qsa_sparse_decode_workspace_bytes(B: int, T: int, Hq: int, Hkv: int, D: int,
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:
-    """Workspace buffer (zero-filled; no call needs it zeroed: the decode
-    zeroes its own header in every call)."""
+    """Workspace buffer (zero-filled; no call needs it zeroed: the stream-K
+    decode keeps no state between calls and the chunked decode zeroes its
+    header in every call)."""
     return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
 
 
